@@ -1,0 +1,457 @@
+// C ABI of the library: argument validation, workspace planning, TMA tensor
+// maps and the launch sequence of one optimizer step. Nothing here allocates
+// or synchronises on the step path; all work is enqueued on the caller's stream.
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "muon_b200.h"
+#include "plan.cuh"
+
+using namespace muon;
+
+namespace {
+
+// ------------------------------------------------------------ process state
+struct DebugState {
+  int fault = 0;
+  double wait_limit_s = 2.0;
+};
+DebugState g_debug;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_mu;
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+};
+DeviceState g_dev[64];
+
+muon_status device_state(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MUON_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return MUON_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MUON_ERR_CUDA;
+    if (ns_gemm_prepare() != cudaSuccess) return MUON_ERR_CUDA;
+    d.ready = true;
+  }
+  *sms = d.sms;
+  return MUON_OK;
+}
+
+// ------------------------------------------------------------ validation
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool dtype_ok(int32_t d) { return d == MUON_F32 || d == MUON_BF16; }
+inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr size_t kHeaderBytes = 4096;  // device status word at offset 0
+
+muon_status check_shape(int64_t count, int64_t rows, int64_t cols) {
+  if (count < 1 || rows < 1 || cols < 1) return MUON_ERR_SHAPE;
+  const int64_t Rp = round_up(rows, kPad), Cp = round_up(cols, kPad);
+  const int64_t rp = rows > cols ? Cp : Rp;
+  // TMA coordinates and tile indices are 32-bit
+  if (count * Rp >= (int64_t(1) << 31) || count * rp >= (int64_t(1) << 31)) return MUON_ERR_SHAPE;
+  if (Rp >= (int64_t(1) << 24) || Cp >= (int64_t(1) << 24)) return MUON_ERR_SHAPE;
+  const int64_t tiles = count * (Rp / kBM) * (Cp / kBN);
+  const int64_t chunks = (Rp * Cp + kChunk - 1) / kChunk;
+  if (tiles >= (int64_t(1) << 30) || count * chunks >= (int64_t(1) << 30)) return MUON_ERR_SHAPE;
+  return MUON_OK;
+}
+
+bool finite(float x) { return std::isfinite(x); }
+
+muon_status check_ns(const muon_hparams* hp) {
+  if (hp->ns_steps < 1 || hp->ns_steps > MUON_MAX_NS_STEPS) return MUON_ERR_HPARAM;
+  for (int i = 0; i < 3 * hp->ns_steps; ++i)
+    if (!finite(hp->coeffs[i])) return MUON_ERR_HPARAM;
+  if (!finite(hp->eps) || hp->eps < 0.0f) return MUON_ERR_HPARAM;
+  return MUON_OK;
+}
+
+inline bool beta_ok(float b) { return finite(b) && b >= 0.0f && b < 1.0f; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+muon_status check_banks(const muon_bank* banks, int32_t nbanks, bool anvil) {
+  if (!banks) return MUON_ERR_NULL;
+  if (nbanks < 1 || nbanks > MUON_MAX_BANKS) return MUON_ERR_SHAPE;
+  for (int b = 0; b < nbanks; ++b) {
+    const muon_bank& k = banks[b];
+    muon_status st = check_shape(k.count, k.rows, k.cols);
+    if (st != MUON_OK) return st;
+    if (!k.param || !k.grad || !k.momentum) return MUON_ERR_NULL;
+    if (anvil && !k.momentum_slow) return MUON_ERR_NULL;
+    if (!dtype_ok(k.param_dtype) || !dtype_ok(k.grad_dtype)) return MUON_ERR_DTYPE;
+    if (!aligned16(k.param) || !aligned16(k.grad) || !aligned16(k.momentum) ||
+        !aligned16(k.momentum_slow) || !aligned16(k.ema))
+      return MUON_ERR_ALIGN;
+    const size_t n = static_cast<size_t>(k.count * k.rows * k.cols);
+    const size_t np = n * (k.param_dtype == MUON_BF16 ? 2 : 4);
+    const void* bufs[4] = {k.param, k.momentum, anvil ? k.momentum_slow : nullptr, k.ema};
+    const size_t sz[4] = {np, n * 4, n * 4, n * 4};
+    for (int i = 0; i < 4; ++i)
+      for (int j = i + 1; j < 4; ++j)
+        if (overlap(bufs[i], sz[i], bufs[j], sz[j])) return MUON_ERR_ALIAS;
+  }
+  return MUON_OK;
+}
+
+// ------------------------------------------------------------ workspace
+struct Shape3 {
+  int64_t count, rows, cols;
+};
+
+// Fills plans (if base != nullptr) and returns the workspace bytes needed.
+size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan* plans) {
+  size_t off = kHeaderBytes;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  for (int b = 0; b < nbanks; ++b) {
+    const Shape3& s = shapes[b];
+    BankPlan p;
+    std::memset(&p, 0, sizeof(p));
+    p.count = static_cast<int>(s.count);
+    p.R = static_cast<int>(s.rows);
+    p.C = static_cast<int>(s.cols);
+    p.Rp = static_cast<int>(round_up(s.rows, kPad));
+    p.Cp = static_cast<int>(round_up(s.cols, kPad));
+    p.tall = s.rows > s.cols ? 1 : 0;
+    p.rp = p.tall ? p.Cp : p.Rp;
+    const size_t padded = static_cast<size_t>(p.Rp) * p.Cp;
+    p.chunks = static_cast<int>((padded + kChunk - 1) / kChunk);
+    const int nb = p.rp / kBN;
+    p.tiles_sym = nb * (nb + 1);
+    p.tiles_apply = (p.Rp / kBM) * (p.Cp / kBN);
+    const size_t it_bytes = static_cast<size_t>(p.count) * padded * 2;
+    const size_t sq_bytes = static_cast<size_t>(p.count) * p.rp * p.rp * 2;
+    const size_t o_hi0 = take(it_bytes), o_hi1 = take(it_bytes), o_lo = take(it_bytes);
+    const size_t o_A = take(sq_bytes), o_B = take(sq_bytes);
+    const size_t o_part = take(static_cast<size_t>(p.count) * p.chunks * 4);
+    const size_t o_scale = take(static_cast<size_t>(p.count) * 4);
+    if (base) {
+      p.hi[0] = reinterpret_cast<__nv_bfloat16*>(base + o_hi0);
+      p.hi[1] = reinterpret_cast<__nv_bfloat16*>(base + o_hi1);
+      p.lo = reinterpret_cast<__nv_bfloat16*>(base + o_lo);
+      p.A = reinterpret_cast<__nv_bfloat16*>(base + o_A);
+      p.B = reinterpret_cast<__nv_bfloat16*>(base + o_B);
+      p.partial = reinterpret_cast<float*>(base + o_part);
+      p.scale = reinterpret_cast<float*>(base + o_scale);
+      plans[b] = p;
+    }
+  }
+  return off;
+}
+
+muon_status encode_map(CUtensorMap* m, void* ptr, int64_t inner, int64_t outer, int box_outer) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MUON_OK : MUON_ERR_CUDA;
+}
+
+muon_status encode_bank_maps(const BankPlan& p, CUtensorMap* maps) {
+  const int64_t rows = static_cast<int64_t>(p.count) * p.Rp;
+  const int64_t srows = static_cast<int64_t>(p.count) * p.rp;
+  muon_status st;
+  for (int k = 0; k < 2; ++k) {
+    if ((st = encode_map(&maps[kHiK0 + k], p.hi[k], p.Cp, rows, 128)) != MUON_OK) return st;
+    if ((st = encode_map(&maps[kHiMN0 + k], p.hi[k], p.Cp, rows, 64)) != MUON_OK) return st;
+  }
+  if ((st = encode_map(&maps[kAK], p.A, p.rp, srows, 128)) != MUON_OK) return st;
+  return encode_map(&maps[kBK_], p.B, p.rp, srows, 128);
+}
+
+// ------------------------------------------------------------ the step
+enum class Variant { kMuon, kAnvil, kOrtho };
+
+struct OrthoIO {
+  const void* in;
+  int in_dtype;
+  void* out;
+  int out_dtype;
+};
+
+muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_hparams* hp,
+                     void* ws, size_t ws_bytes, cudaStream_t stream, const OrthoIO* oio) {
+  int sms = 0;
+  muon_status st = device_state(&sms);
+  if (st != MUON_OK) return st;
+
+  Shape3 shapes[MUON_MAX_BANKS];
+  for (int b = 0; b < nbanks; ++b) shapes[b] = {banks[b].count, banks[b].rows, banks[b].cols};
+  static thread_local NsGemmParams gp;  // large; kept off the stack
+  std::memset(&gp, 0, sizeof(gp));
+  BankPlan plans[MUON_MAX_BANKS];
+  const size_t need = plan_workspace(shapes, nbanks, static_cast<uint8_t*>(ws), plans);
+  if (ws_bytes < need) return MUON_ERR_WORKSPACE;
+  int* status = static_cast<int*>(ws);
+
+  // ---- momentum + norm partials, then 1/(||U||+eps)
+  MomParams mp;
+  std::memset(&mp, 0, sizeof(mp));
+  mp.nbanks = nbanks;
+  mp.mode = v == Variant::kMuon ? kMomMuon : (v == Variant::kAnvil ? kMomAnvil : kMomNone);
+  mp.mu = v == Variant::kAnvil ? hp->beta_fast : hp->mu;
+  mp.mu_slow = hp->beta_slow;
+  mp.nesterov = hp->nesterov ? 1 : 0;
+  mp.eps = hp->eps;
+  int blocks = 0, mats = 0;
+  for (int b = 0; b < nbanks; ++b) {
+    mp.bank[b] = plans[b];
+    if (v == Variant::kOrtho) {
+      mp.io[b] = {oio->in, nullptr, nullptr, oio->in_dtype};
+    } else {
+      mp.io[b] = {banks[b].grad, banks[b].momentum, banks[b].momentum_slow, banks[b].grad_dtype};
+    }
+    mp.block_begin[b] = blocks;
+    mp.mat_begin[b] = mats;
+    blocks += plans[b].count * plans[b].chunks;
+    mats += plans[b].count;
+  }
+  mp.block_begin[nbanks] = blocks;
+  mp.mat_begin[nbanks] = mats;
+  if (launch_momentum_norm(mp, blocks, mats, stream) != cudaSuccess) return MUON_ERR_CUDA;
+
+  // ---- Newton-Schulz chain
+  gp.nbanks = nbanks;
+  gp.status = status;
+  const double lim = g_debug.wait_limit_s > 0 ? g_debug.wait_limit_s : 2.0;
+  gp.wait_limit_ns = static_cast<unsigned long long>(lim * 1e9);
+  gp.fault = g_debug.fault;
+  for (int b = 0; b < nbanks; ++b) {
+    gp.bank[b] = plans[b];
+    if ((st = encode_bank_maps(plans[b], gp.maps[b])) != MUON_OK) return st;
+  }
+  for (int it = 0; it < hp->ns_steps; ++it) {
+    gp.iter = it;
+    gp.cur = it & 1;
+    gp.a = hp->coeffs[3 * it];
+    gp.b = hp->coeffs[3 * it + 1];
+    gp.c = hp->coeffs[3 * it + 2];
+    for (int ph = kGram; ph <= kApply; ++ph) {
+      gp.phase = ph;
+      int tiles = 0;
+      for (int b = 0; b < nbanks; ++b) {
+        gp.tile_begin[b] = tiles;
+        tiles += plans[b].count * (ph == kApply ? plans[b].tiles_apply : plans[b].tiles_sym);
+      }
+      gp.tile_begin[nbanks] = tiles;
+      const int grid = tiles < sms ? tiles : sms;
+      if (launch_ns_gemm(gp, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    }
+  }
+
+  // ---- scale, decay, parameter write (+ EMA), or O out
+  UpdParams up;
+  std::memset(&up, 0, sizeof(up));
+  up.nbanks = nbanks;
+  up.mode = v == Variant::kMuon ? kUpdDecoupled : (v == Variant::kAnvil ? kUpdCautious : kUpdWriteO);
+  up.final_buf = hp->ns_steps & 1;
+  up.lr_wd = hp->lr * hp->weight_decay;
+  up.ema_beta = hp->ema_beta;
+  long long total = 0;
+  for (int b = 0; b < nbanks; ++b) {
+    up.bank[b] = plans[b];
+    const double s = std::sqrt(std::fmax(1.0, double(banks[b].rows) / double(banks[b].cols)));
+    if (v == Variant::kOrtho) {
+      up.io[b] = {oio->out, oio->out_dtype, nullptr, nullptr, 0.0f};
+    } else {
+      up.io[b] = {banks[b].param, banks[b].param_dtype, banks[b].momentum_slow, banks[b].ema,
+                  static_cast<float>(double(hp->lr) * s)};
+    }
+    up.elem_begin[b] = total;
+    total += static_cast<long long>(banks[b].count) * banks[b].rows * banks[b].cols;
+  }
+  up.elem_begin[nbanks] = total;
+  if (launch_update(up, total, sms, stream) != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+muon_status check_common(const muon_bank* banks, int32_t nbanks, const muon_hparams* hp, void* ws,
+                         bool anvil) {
+  if (!hp) return MUON_ERR_NULL;
+  muon_status st = check_banks(banks, nbanks, anvil);
+  if (st != MUON_OK) return st;
+  if ((st = check_ns(hp)) != MUON_OK) return st;
+  if (!finite(hp->lr) || !finite(hp->weight_decay) || hp->weight_decay < 0.0f) return MUON_ERR_HPARAM;
+  if (anvil) {
+    if (!beta_ok(hp->beta_fast) || !beta_ok(hp->beta_slow)) return MUON_ERR_HPARAM;
+  } else if (!beta_ok(hp->mu)) {
+    return MUON_ERR_HPARAM;
+  }
+  for (int b = 0; b < nbanks; ++b)
+    if (banks[b].ema && !beta_ok(hp->ema_beta)) return MUON_ERR_HPARAM;
+  if (!ws) return MUON_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MUON_ERR_ALIGN;
+  return MUON_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t muon_abi_version(void) { return MUON_ABI_VERSION; }
+
+const char* muon_status_string(muon_status s) {
+  switch (s) {
+    case MUON_OK: return "MUON_OK";
+    case MUON_ERR_NULL: return "MUON_ERR_NULL: a required pointer is NULL";
+    case MUON_ERR_SHAPE: return "MUON_ERR_SHAPE: bad count/rows/cols or number of banks";
+    case MUON_ERR_DTYPE: return "MUON_ERR_DTYPE: unsupported dtype";
+    case MUON_ERR_ALIGN: return "MUON_ERR_ALIGN: pointer not 16-byte aligned";
+    case MUON_ERR_HPARAM: return "MUON_ERR_HPARAM: hyper-parameter out of range";
+    case MUON_ERR_WORKSPACE: return "MUON_ERR_WORKSPACE: workspace missing or too small";
+    case MUON_ERR_CUDA: return "MUON_ERR_CUDA: CUDA runtime error";
+    case MUON_ERR_TIMEOUT: return "MUON_ERR_TIMEOUT: a bounded device wait ran out";
+    case MUON_ERR_ALIAS: return "MUON_ERR_ALIAS: in-place buffers overlap";
+  }
+  return "unknown muon_status";
+}
+
+size_t muon_workspace_size(const muon_bank* banks, int32_t nbanks) {
+  if (!banks || nbanks < 1 || nbanks > MUON_MAX_BANKS) return 0;
+  Shape3 shapes[MUON_MAX_BANKS];
+  for (int b = 0; b < nbanks; ++b) {
+    if (check_shape(banks[b].count, banks[b].rows, banks[b].cols) != MUON_OK) return 0;
+    shapes[b] = {banks[b].count, banks[b].rows, banks[b].cols};
+  }
+  return plan_workspace(shapes, nbanks, nullptr, nullptr);
+}
+
+muon_status muon_step(const muon_bank* banks, int32_t nbanks, const muon_hparams* hp, void* ws,
+                      size_t ws_bytes, void* stream) {
+  muon_status st = check_common(banks, nbanks, hp, ws, false);
+  if (st != MUON_OK) return st;
+  if (ws_bytes < muon_workspace_size(banks, nbanks)) return MUON_ERR_WORKSPACE;
+  return run_step(Variant::kMuon, banks, nbanks, hp, ws, ws_bytes,
+                  static_cast<cudaStream_t>(stream), nullptr);
+}
+
+muon_status anvil_step(const muon_bank* banks, int32_t nbanks, const muon_hparams* hp, void* ws,
+                       size_t ws_bytes, void* stream) {
+  muon_status st = check_common(banks, nbanks, hp, ws, true);
+  if (st != MUON_OK) return st;
+  if (ws_bytes < muon_workspace_size(banks, nbanks)) return MUON_ERR_WORKSPACE;
+  return run_step(Variant::kAnvil, banks, nbanks, hp, ws, ws_bytes,
+                  static_cast<cudaStream_t>(stream), nullptr);
+}
+
+muon_status muon_orthogonalize(const void* in, int32_t in_dtype, void* out, int32_t out_dtype,
+                               int64_t count, int64_t rows, int64_t cols, const muon_hparams* hp,
+                               void* ws, size_t ws_bytes, void* stream) {
+  if (!in || !out || !hp) return MUON_ERR_NULL;
+  muon_status st = check_shape(count, rows, cols);
+  if (st != MUON_OK) return st;
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return MUON_ERR_DTYPE;
+  if (!aligned16(in) || !aligned16(out)) return MUON_ERR_ALIGN;
+  if ((st = check_ns(hp)) != MUON_OK) return st;
+  if (!ws) return MUON_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MUON_ERR_ALIGN;
+  muon_bank bank;
+  std::memset(&bank, 0, sizeof(bank));
+  bank.count = count;
+  bank.rows = rows;
+  bank.cols = cols;
+  if (ws_bytes < muon_workspace_size(&bank, 1)) return MUON_ERR_WORKSPACE;
+  const size_t n = static_cast<size_t>(count * rows * cols);
+  if (overlap(in, n * (in_dtype == MUON_BF16 ? 2 : 4), out, n * (out_dtype == MUON_BF16 ? 2 : 4)))
+    return MUON_ERR_ALIAS;
+  OrthoIO io{in, in_dtype, out, out_dtype};
+  return run_step(Variant::kOrtho, &bank, 1, hp, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                  &io);
+}
+
+muon_status ema_update(const muon_bank* banks, int32_t nbanks, float beta, void* stream) {
+  if (!banks) return MUON_ERR_NULL;
+  if (nbanks < 1 || nbanks > MUON_MAX_BANKS) return MUON_ERR_SHAPE;
+  if (!beta_ok(beta)) return MUON_ERR_HPARAM;
+  for (int b = 0; b < nbanks; ++b) {
+    const muon_bank& k = banks[b];
+    if (!k.ema) continue;
+    if (k.count < 1 || k.rows < 1 || k.cols < 1) return MUON_ERR_SHAPE;
+    if (!k.param) return MUON_ERR_NULL;
+    if (!dtype_ok(k.param_dtype)) return MUON_ERR_DTYPE;
+    if (!aligned16(k.param) || !aligned16(k.ema)) return MUON_ERR_ALIGN;
+  }
+  int sms = 0;
+  muon_status st = device_state(&sms);
+  if (st != MUON_OK) return st;
+  for (int b = 0; b < nbanks; ++b) {
+    const muon_bank& k = banks[b];
+    if (!k.ema) continue;
+    if (launch_ema(k.ema, k.param, k.param_dtype, k.count * k.rows * k.cols, beta, sms,
+                   static_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return MUON_ERR_CUDA;
+  }
+  return MUON_OK;
+}
+
+muon_status readout_blend(const void* theta, int32_t theta_dtype, const float* ema, void* out,
+                          int32_t out_dtype, int64_t n, float w_final, void* stream) {
+  if (!theta || !ema || !out) return MUON_ERR_NULL;
+  if (n < 1) return MUON_ERR_SHAPE;
+  if (!dtype_ok(theta_dtype) || !dtype_ok(out_dtype)) return MUON_ERR_DTYPE;
+  if (!aligned16(theta) || !aligned16(ema) || !aligned16(out)) return MUON_ERR_ALIGN;
+  if (!finite(w_final)) return MUON_ERR_HPARAM;
+  int sms = 0;
+  muon_status st = device_state(&sms);
+  if (st != MUON_OK) return st;
+  if (launch_blend(theta, theta_dtype, ema, out, out_dtype, n, w_final, sms,
+                   static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  return MUON_OK;
+}
+
+muon_status muon_device_status(void* ws, size_t ws_bytes, void* stream, int32_t clear) {
+  if (!ws) return MUON_ERR_NULL;
+  if (ws_bytes < kHeaderBytes) return MUON_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MUON_ERR_CUDA;
+  if (clear) {
+    if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return MUON_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MUON_ERR_CUDA;
+  }
+  return v == 0 ? MUON_OK : static_cast<muon_status>(v);
+}
+
+muon_status muon_set_debug(int32_t fault_mode, double wait_limit_seconds) {
+  if (fault_mode < 0 || fault_mode > 1) return MUON_ERR_HPARAM;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_debug.fault = fault_mode;
+  g_debug.wait_limit_s = wait_limit_seconds > 0 ? wait_limit_seconds : 2.0;
+  return MUON_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,374 @@
+// Newton-Schulz GEMM chain on sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One persistent launch per (step, phase). The three phases of a step are
+//   Gram : A = X X^T            (tall: A = Y^T Y)      upper tiles only, mirrored
+//   Poly : B = b A + c A A      (A symmetric)          upper tiles only, mirrored
+//   Apply: X <- a X + B X       (tall: Y <- a Y + Y B) full tiles
+// ("Muonとは" / "Muonが登場": approximate orthogonalisation by Newton-Schulz
+// iteration, bf16 operands; the polynomial step is the method statement's).
+//
+// Block layout (192 threads, one block per SM):
+//   warp 0     one thread issues TMA loads into a 4-stage smem ring
+//   warp 1     allocates 512 TMEM columns; one thread issues tcgen05.mma
+//              (M=128, N=256, K=16, bf16 in, fp32 accumulate) into one of two
+//              256-column accumulators
+//   warps 2..5 epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
+//              32*(w%4)..+31, i.e. tile rows), apply the phase's axpy and store
+// Tiles are 128 x 256 with K in 64-element (128-byte, swizzled) steps. The
+// epilogue of tile t overlaps the MMAs of tile t+1 through the two
+// accumulators. Every wait is bounded (muon::mbar_wait).
+#include <cuda_runtime.h>
+
+#include "plan.cuh"
+#include "ptx.cuh"
+
+namespace muon {
+
+struct Tile {
+  int bank, mat, m0, n0, nkb;
+  int a_map, a_mn, a_base;
+  int b_map, b_mn, b_base;
+};
+
+// Upper tiles of a symmetric product with 2*nb row blocks (128) and nb column
+// blocks (256): row blocks 2p and 2p+1 hold column blocks p .. nb-1.
+__device__ __forceinline__ void sym_tile(int t, int nb, int& i, int& j) {
+  int p = 0;
+  for (;;) {
+    const int cnt = 2 * (nb - p);
+    if (t < cnt) break;
+    t -= cnt;
+    ++p;
+  }
+  const int per = nb - p;
+  i = 2 * p + t / per;
+  j = p + t % per;
+}
+
+__device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
+  Tile T;
+  int b = 0;
+  while (b + 1 < p.nbanks && tile >= p.tile_begin[b + 1]) ++b;
+  const BankPlan& bp = p.bank[b];
+  const int local = tile - p.tile_begin[b];
+  T.bank = b;
+  if (p.phase == kApply) {
+    T.mat = local / bp.tiles_apply;
+    const int t = local - T.mat * bp.tiles_apply;
+    const int nbn = bp.Cp / kBN;
+    T.m0 = (t / nbn) * kBM;
+    T.n0 = (t % nbn) * kBN;
+  } else {
+    T.mat = local / bp.tiles_sym;
+    const int t = local - T.mat * bp.tiles_sym;
+    int i, j;
+    sym_tile(t, bp.rp / kBN, i, j);
+    T.m0 = i * kBM;
+    T.n0 = j * kBN;
+  }
+  const int cur = p.cur;
+  const int xbase = T.mat * bp.Rp;   // first row of this matrix in the iterate maps
+  const int sbase = T.mat * bp.rp;   // first row of this matrix in the A / B maps
+  if (p.phase == kGram) {
+    if (!bp.tall) {  // D[m][n] = sum_k X[m][k] X[n][k]
+      T.a_map = kHiK0 + cur; T.a_mn = 0; T.a_base = xbase;
+      T.b_map = kHiK0 + cur; T.b_mn = 0; T.b_base = xbase;
+      T.nkb = bp.Cp / kBK;
+    } else {         // D[m][n] = sum_k Y[k][m] Y[k][n]
+      T.a_map = kHiMN0 + cur; T.a_mn = 1; T.a_base = xbase;
+      T.b_map = kHiMN0 + cur; T.b_mn = 1; T.b_base = xbase;
+      T.nkb = bp.Rp / kBK;
+    }
+  } else if (p.phase == kPoly) {  // D[m][n] = sum_k A[m][k] A[n][k]
+    T.a_map = kAK; T.a_mn = 0; T.a_base = sbase;
+    T.b_map = kAK; T.b_mn = 0; T.b_base = sbase;
+    T.nkb = bp.rp / kBK;
+  } else {
+    if (!bp.tall) {  // D[m][n] = sum_k B[m][k] X[k][n]
+      T.a_map = kBK_; T.a_mn = 0; T.a_base = sbase;
+      T.b_map = kHiMN0 + cur; T.b_mn = 1; T.b_base = xbase;
+      T.nkb = bp.Rp / kBK;
+    } else {         // D[m][n] = sum_k Y[m][k] B[n][k]
+      T.a_map = kHiK0 + cur; T.a_mn = 0; T.a_base = xbase;
+      T.b_map = kBK_; T.b_mn = 0; T.b_base = sbase;
+      T.nkb = bp.Cp / kBK;
+    }
+  }
+  return T;
+}
+
+// One operand tile of `rows` (MN extent) x 64 (K) into dst.
+//  K-major : boxes of 128 rows x 64 K (16 KB), stacked along MN.
+//  MN-major: boxes of 64 K rows x 64 MN (8 KB), stacked along MN.
+__device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                             int mn_major, int rows, int base, int mn0, int k0) {
+  if (!mn_major) {
+    for (int i = 0; i < rows / 128; ++i)
+      tma_load_2d(dst + i * 16384, map, bar, k0, base + mn0 + 128 * i);
+  } else {
+    for (int j = 0; j < rows / 64; ++j)
+      tma_load_2d(dst + j * 8192, map, bar, mn0 + 64 * j, base + k0);
+  }
+}
+
+__device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_major, int ks) {
+  return mn_major ? smem_desc_sw128(tile_addr + ks * 2048, 8192, 1024)
+                  : smem_desc_sw128(tile_addr + ks * 32, 16, 1024);
+}
+
+// ---------------------------------------------------------------- epilogues
+// Gram / Poly: row `row` of the tile, columns col0 .. col0+31 in v[]. Stores
+// the upper part (col >= row) in place and mirrors the strict upper part.
+__device__ __forceinline__ void epilogue_sym(const NsGemmParams& p, const BankPlan& bp, int mat,
+                                             int row, int col0, float (&v)[32]) {
+  if (col0 + 31 < row) return;  // entirely below the diagonal: the mirror covers it
+  const size_t rp = static_cast<size_t>(bp.rp);
+  const size_t mbase = static_cast<size_t>(mat) * rp * rp;
+  __nv_bfloat16* out = (p.phase == kGram ? bp.A : bp.B) + mbase;
+  if (p.phase == kGram) {
+    if (p.iter == 0) {  // the operand holds U; fold 1 / ||U||^2 in here
+      const float s = bp.scale[mat];
+      const float s2 = s * s;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) v[t] *= s2;
+    }
+  } else {
+    const uint4* ain = reinterpret_cast<const uint4*>(bp.A + mbase + row * rp + col0);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint4 w = ain[g];
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        v[8 * g + 2 * h] = fmaf(p.c, v[8 * g + 2 * h], p.b * bf16_lo_f(ww[h]));
+        v[8 * g + 2 * h + 1] = fmaf(p.c, v[8 * g + 2 * h + 1], p.b * bf16_hi_f(ww[h]));
+      }
+    }
+  }
+  uint32_t pk[16];
+#pragma unroll
+  for (int h = 0; h < 16; ++h) pk[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
+  __nv_bfloat16* orow = out + row * rp + col0;
+  if (col0 >= row) {
+    uint4* o4 = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) o4[g] = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+  } else {
+    const unsigned short* ps = reinterpret_cast<const unsigned short*>(pk);
+#pragma unroll
+    for (int t = 0; t < 32; ++t)
+      if (col0 + t >= row) reinterpret_cast<unsigned short*>(orow)[t] = ps[t];
+  }
+  const unsigned short* ps = reinterpret_cast<const unsigned short*>(pk);
+  unsigned short* ocol = reinterpret_cast<unsigned short*>(out + static_cast<size_t>(col0) * rp + row);
+#pragma unroll
+  for (int t = 0; t < 32; ++t)
+    if (col0 + t > row) ocol[static_cast<size_t>(t) * rp] = ps[t];
+}
+
+// Apply: x' = alpha x + beta D with x = hi + lo; writes hi' (other buffer) and lo.
+__device__ __forceinline__ void epilogue_apply(const NsGemmParams& p, const BankPlan& bp, int mat,
+                                               int row, int col0, const float (&v)[32]) {
+  const size_t off = static_cast<size_t>(mat) * bp.Rp * bp.Cp + static_cast<size_t>(row) * bp.Cp + col0;
+  const uint4* hin = reinterpret_cast<const uint4*>(bp.hi[p.cur] + off);
+  uint4* hout = reinterpret_cast<uint4*>(bp.hi[p.cur ^ 1] + off);
+  uint4* lio = reinterpret_cast<uint4*>(bp.lo + off);
+  float alpha = p.a, beta = 1.0f;
+  if (p.iter == 0) {  // the iterate holds U; X0 = s U
+    const float s = bp.scale[mat];
+    alpha *= s;
+    beta = s;
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const uint4 h4 = hin[g];
+    const uint4 l4 = lio[g];
+    const uint32_t hw[4] = {h4.x, h4.y, h4.z, h4.w};
+    const uint32_t lw[4] = {l4.x, l4.y, l4.z, l4.w};
+    uint32_t ho[4], lo[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float x0 = bf16_lo_f(hw[h]) + bf16_lo_f(lw[h]);
+      const float x1 = bf16_hi_f(hw[h]) + bf16_hi_f(lw[h]);
+      const float y0 = fmaf(alpha, x0, beta * v[8 * g + 2 * h]);
+      const float y1 = fmaf(alpha, x1, beta * v[8 * g + 2 * h + 1]);
+      ho[h] = pack_bf16x2(y0, y1);
+      lo[h] = pack_bf16x2(y0 - bf16_lo_f(ho[h]), y1 - bf16_hi_f(ho[h]));
+    }
+    hout[g] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+    lio[g] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
+// Waits that ignore the abort flag, used only to drain in-flight work.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(addr, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return;
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ NsGemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t limit = p.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int b = 0; b < p.nbanks; ++b)
+      for (int k = 0; k < kMaxMaps; ++k) tma_prefetch_map(&p.maps[b][k]);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued_parity[kStages];
+      for (int s = 0; s < kStages; ++s) issued_parity[s] = -1;
+      bool ok = true;
+      bool first = true;
+      for (int tile = blockIdx.x; ok && tile < p.tile_begin[p.nbanks]; tile += gridDim.x) {
+        const Tile T = decode_tile(p, tile);
+        const CUtensorMap* amap = &p.maps[T.bank][T.a_map];
+        const CUtensorMap* bmap = &p.maps[T.bank][T.b_map];
+        for (int kb = 0; kb < T.nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, limit)) { ok = false; break; }
+          const bool withhold = first && p.fault == 1 && blockIdx.x == 0;
+          first = false;
+          if (!withhold) {
+            uint8_t* st = tiles + stage * kStageBytes;
+            mbar_arrive_expect_tx(&full[stage], kStageBytes);
+            load_operand(st, amap, &full[stage], T.a_mn, kBM, T.a_base, T.m0, kb * kBK);
+            load_operand(st + kATileBytes, bmap, &full[stage], T.b_mn, kBN, T.b_base, T.n0, kb * kBK);
+            issued_parity[stage] = static_cast<int>(phase);
+          }
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // make sure no bulk copy is still landing in shared memory
+      for (int s = 0; s < kStages; ++s)
+        if (issued_parity[s] >= 0) drain_wait(&full[s], static_cast<uint32_t>(issued_parity[s]), limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.tile_begin[p.nbanks]; tile += gridDim.x) {
+        const Tile T = decode_tile(p, tile);
+        const uint32_t idesc = idesc_bf16(kBM, kBN, T.a_mn, T.b_mn);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, limit)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        for (int kb = 0; kb < T.nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, limit)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(tiles + stage * kStageBytes);
+          const uint32_t b_addr = a_addr + kATileBytes;
+#pragma unroll
+          for (int ks = 0; ks < kBK / 16; ++ks) {
+            umma_bf16(d_tmem, operand_desc(a_addr, T.a_mn, ks), operand_desc(b_addr, T.b_mn, ks),
+                      idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // every MMA issued by this thread has finished before TMEM is released
+      umma_commit(done);
+      drain_wait(done, 0, limit);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.tile_begin[p.nbanks]; tile += gridDim.x) {
+      const Tile T = decode_tile(p, tile);
+      // the tcgen05.ld below is warp-collective: leave only if the whole warp does
+      const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, limit);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const BankPlan& bp = p.bank[T.bank];
+      const int row = T.m0 + 32 * q + lane;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * kBN);
+      for (int j = 0; j < kBN / 32; ++j) {
+        uint32_t r[32];
+        tmem_ld32(tb + 32 * j, r);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+        if (p.phase == kApply)
+          epilogue_apply(p, bp, T.mat, row, T.n0 + 32 * j, v);
+        else
+          epilogue_sym(p, bp, T.mat, row, T.n0 + 32 * j, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+cudaError_t ns_gemm_prepare() {
+  return cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kGemmSmemBytes);
+}
+
+cudaError_t launch_ns_gemm(const NsGemmParams& p, int grid, cudaStream_t s) {
+  ns_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

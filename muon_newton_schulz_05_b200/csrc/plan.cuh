@@ -1,0 +1,123 @@
+// Internal plan structures shared by the host API and the kernels.
+//
+// Working layout. Every matrix keeps the layout of its momentum, R x C
+// row-major, padded with zeros to Rp x Cp (multiples of 256). A wide matrix
+// (R <= C) is iterated as X (r = R): A = X X^T, X <- aX + BX. A tall matrix
+// (R > C) is iterated as Y = X^T in the same storage: A = Y^T Y (r = C),
+// Y <- aY + Y B (B symmetric). Nothing is ever transposed in memory; the GEMMs
+// read the operands K-major or MN-major instead. Zero padding is exact: the
+// padded rows and columns of X, A and B stay exactly zero through the
+// iteration, because the polynomial is odd.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "muon_b200.h"
+
+namespace muon {
+
+constexpr int kPad = 256;          // padding granule of R and C
+constexpr int kBM = 128;           // GEMM tile rows (UMMA M)
+constexpr int kBN = 256;           // GEMM tile cols (UMMA N)
+constexpr int kBK = 64;            // K per pipeline stage (one 128-byte swizzle row)
+constexpr int kStages = 4;         // TMA -> MMA pipeline depth
+constexpr int kATileBytes = kBM * kBK * 2;
+constexpr int kBTileBytes = kBN * kBK * 2;
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kChunk = 8192;       // padded elements per block in the momentum pass
+constexpr int kMaxMaps = 6;
+
+enum Phase : int { kGram = 0, kPoly = 1, kApply = 2 };
+
+// Tensor-map slots per bank.
+enum MapSlot : int { kHiK0 = 0, kHiK1 = 1, kHiMN0 = 2, kHiMN1 = 3, kAK = 4, kBK_ = 5 };
+
+struct BankPlan {
+  int count, R, C, Rp, Cp, rp, tall;
+  int chunks;                   // momentum-pass blocks per matrix
+  int tiles_sym;                // upper tiles of an rp x rp symmetric product
+  int tiles_apply;              // (Rp/128) * (Cp/256)
+  __nv_bfloat16* hi[2];         // iterate, high bf16 part (ping-pong)
+  __nv_bfloat16* lo;            // iterate, low bf16 part (in place)
+  __nv_bfloat16* A;             // Gram matrix, count x rp x rp
+  __nv_bfloat16* B;             // b A + c A^2, count x rp x rp
+  float* partial;               // count x chunks sums of squares
+  float* scale;                 // count: 1 / (||U||_F + eps)
+};
+
+// ---------------------------------------------------------------- GEMM chain
+struct NsGemmParams {
+  CUtensorMap maps[MUON_MAX_BANKS][kMaxMaps];
+  BankPlan bank[MUON_MAX_BANKS];
+  int tile_begin[MUON_MAX_BANKS + 1];
+  int nbanks;
+  int phase;          // Phase
+  int iter;           // 0-based Newton-Schulz step
+  int cur;            // hi buffer holding the current iterate
+  float a, b, c;      // this step's coefficients
+  int* status;        // device status word
+  unsigned long long wait_limit_ns;
+  int fault;          // test hook (muon_set_debug)
+};
+
+// ---------------------------------------------------------- momentum + norm
+struct MomBank {
+  const void* grad;
+  float* mom;
+  float* mom_slow;
+  int grad_dtype;
+};
+
+enum MomMode : int { kMomMuon = 0, kMomAnvil = 1, kMomNone = 2 };
+
+struct MomParams {
+  BankPlan bank[MUON_MAX_BANKS];
+  MomBank io[MUON_MAX_BANKS];
+  int block_begin[MUON_MAX_BANKS + 1];
+  int nbanks;
+  int mode;           // MomMode
+  float mu;           // Muon mu, or ANVIL beta_fast
+  float mu_slow;      // ANVIL beta_slow
+  int nesterov;
+  float eps;
+  int mat_begin[MUON_MAX_BANKS + 1];
+};
+
+// --------------------------------------------------------------- update pass
+enum UpdMode : int { kUpdDecoupled = 0, kUpdCautious = 1, kUpdWriteO = 2 };
+
+struct UpdBank {
+  void* param;          // param (or O output in kUpdWriteO)
+  int param_dtype;
+  const float* mom_slow;
+  float* ema;
+  float step_scale;     // lr * max(1, R/C)^(1/2)
+};
+
+struct UpdParams {
+  BankPlan bank[MUON_MAX_BANKS];
+  UpdBank io[MUON_MAX_BANKS];
+  long long elem_begin[MUON_MAX_BANKS + 1];   // logical elements, prefix sums
+  int nbanks;
+  int mode;
+  int final_buf;        // hi buffer holding the last iterate
+  float lr_wd;          // lr * weight_decay
+  float ema_beta;
+};
+
+// Launchers (defined in the .cu files).
+cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total_mats,
+                                 cudaStream_t s);
+cudaError_t launch_ns_gemm(const NsGemmParams& p, int grid, cudaStream_t s);
+cudaError_t launch_update(const UpdParams& p, long long total_elems, int num_sms,
+                          cudaStream_t s);
+cudaError_t launch_ema(float* ema, const void* param, int param_dtype, long long n, float beta,
+                       int num_sms, cudaStream_t s);
+cudaError_t launch_blend(const void* theta, int theta_dtype, const float* ema, void* out,
+                         int out_dtype, long long n, float w_final, int num_sms, cudaStream_t s);
+cudaError_t ns_gemm_prepare();   // one-time function attributes
+
+}  // namespace muon

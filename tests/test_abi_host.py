@@ -1,0 +1,160 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library loads on a machine without a GPU (the CUDA runtime is linked
+statically and only touched after argument validation), so every validation
+path and the workspace planner can be exercised here.
+"""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import muon_newton_schulz_05_b200 as mb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muon_b200.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(mb.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(mb.EXPORTED) == names
+
+
+def test_version_and_strings():
+    assert mb.abi_version() == 1
+    for code, name in mb.STATUS_NAMES.items():
+        assert mb.status_string(code).startswith(name)
+    assert "unknown" in mb.status_string(77)
+
+
+def test_struct_layout_matches_header():
+    """Compile a probe against the header with gcc and compare with ctypes."""
+    probe = r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "muon_b200.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(muon_bank), offsetof(muon_bank, grad),
+         offsetof(muon_bank, ema), sizeof(muon_hparams), offsetof(muon_hparams, coeffs),
+         offsetof(muon_hparams, beta_slow));
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "p.c")
+        exe = os.path.join(d, "p")
+        open(c, "w").write(probe)
+        subprocess.check_call(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), c, "-o", exe])
+        got = [int(x) for x in subprocess.check_output([exe]).split()]
+    want = [ctypes.sizeof(mb.CBank), mb.CBank.grad.offset, mb.CBank.ema.offset,
+            ctypes.sizeof(mb.CHparams), mb.CHparams.coeffs.offset, mb.CHparams.beta_slow.offset]
+    assert got == want
+
+
+def test_workspace_size_planning():
+    s1 = mb.workspace_size([(1, 256, 512)])
+    # 3 iterate buffers 256x512 bf16, A and B 256^2 bf16, header and small arrays
+    assert s1 >= 3 * 256 * 512 * 2 + 2 * 256 * 256 * 2
+    assert mb.workspace_size([(2, 256, 512)]) > s1
+    # padding to multiples of 256 in both directions
+    assert mb.workspace_size([(1, 7, 13)]) == mb.workspace_size([(1, 256, 256)])
+    # tall and wide banks share the Gram size
+    assert mb.workspace_size([(3, 768, 3072)]) == mb.workspace_size([(3, 3072, 768)])
+    assert mb.workspace_size([(0, 4, 4)]) == 0
+    assert mb.workspace_size([(1, 0, 4)]) == 0
+    assert mb.workspace_size([]) == 0
+    assert mb.workspace_size([(1, 8, 8)] * 9) == 0  # more than MUON_MAX_BANKS
+
+
+FAKE = 0x10000  # aligned, never dereferenced: validation fails first
+
+
+def _bank(**kw):
+    b = mb.CBank()
+    b.count, b.rows, b.cols = kw.get("count", 1), kw.get("rows", 8), kw.get("cols", 8)
+    b.param = kw.get("param", FAKE)
+    b.param_dtype = kw.get("param_dtype", mb.BF16)
+    b.grad = kw.get("grad", FAKE + 0x1000)
+    b.grad_dtype = kw.get("grad_dtype", mb.BF16)
+    b.momentum = kw.get("momentum", FAKE + 0x2000)
+    b.momentum_slow = kw.get("momentum_slow", None)
+    b.ema = kw.get("ema", None)
+    return b
+
+
+def _call(fn, bank, hp=None, ws=FAKE * 16, ws_bytes=1 << 30, nb=1):
+    lib = mb.raw_library()
+    arr = (mb.CBank * 1)(bank)
+    h = (hp or mb.Hparams()).to_c()
+    return getattr(lib, fn)(arr, nb, ctypes.byref(h), ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("fn", ["muon_step", "anvil_step"])
+def test_validation_paths(fn):
+    anvil = fn == "anvil_step"
+    slow = FAKE + 0x3000 if anvil else None
+    ok = dict(momentum_slow=slow)
+    lib = mb.raw_library()
+    h = mb.Hparams().to_c()
+    assert getattr(lib, fn)(None, 1, ctypes.byref(h), FAKE, 1 << 30, None) == 1
+    assert _call(fn, _bank(**ok), nb=0) == 2
+    assert _call(fn, _bank(count=0, **ok)) == 2
+    assert _call(fn, _bank(rows=-3, **ok)) == 2
+    assert _call(fn, _bank(param=None, **ok)) == 1
+    assert _call(fn, _bank(grad=None, **ok)) == 1
+    assert _call(fn, _bank(param_dtype=5, **ok)) == 3
+    assert _call(fn, _bank(grad=FAKE + 0x1004, **ok)) == 4
+    assert _call(fn, _bank(**ok), hp=mb.Hparams(coeffs=[])) == 5
+    assert _call(fn, _bank(**ok), hp=mb.Hparams(coeffs=[(1, 0, 0)] * 17)) == 5
+    assert _call(fn, _bank(**ok), hp=mb.Hparams(coeffs=[(float("nan"), 0, 0)])) == 5
+    assert _call(fn, _bank(**ok), hp=mb.Hparams(eps=-1.0)) == 5
+    assert _call(fn, _bank(**ok), ws=None) == 6
+    assert _call(fn, _bank(**ok), ws_bytes=1024) == 6
+    assert _call(fn, _bank(param=FAKE, momentum=FAKE + 16, **ok)) == 9
+    if anvil:
+        assert _call(fn, _bank()) == 1  # momentum_slow missing
+        assert _call(fn, _bank(**ok), hp=mb.Hparams(beta_slow=1.0)) == 5
+    else:
+        assert _call(fn, _bank(), hp=mb.Hparams(mu=1.5)) == 5
+        assert _call(fn, _bank(ema=FAKE + 0x4000), hp=mb.Hparams(ema_beta=1.0)) == 5
+
+
+def test_valid_call_without_gpu_reports_cuda_error():
+    """All arguments valid: the first CUDA call fails cleanly on a CPU host."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _call("muon_step", _bank()) == 7
+
+
+def test_other_entry_points_validate():
+    lib = mb.raw_library()
+    h = mb.Hparams().to_c()
+    assert lib.muon_orthogonalize(None, 1, FAKE, 1, 1, 8, 8, ctypes.byref(h), FAKE, 1 << 30, None) == 1
+    assert lib.muon_orthogonalize(FAKE, 1, FAKE * 2, 1, 1, 0, 8, ctypes.byref(h), FAKE, 1 << 30, None) == 2
+    assert lib.muon_orthogonalize(FAKE, 7, FAKE * 2, 1, 1, 8, 8, ctypes.byref(h), FAKE, 1 << 30, None) == 3
+    assert lib.muon_orthogonalize(FAKE, 1, FAKE + 2, 1, 1, 8, 8, ctypes.byref(h), FAKE, 1 << 30, None) == 4
+    assert lib.muon_orthogonalize(FAKE, 1, FAKE * 2, 1, 1, 8, 8, ctypes.byref(h), FAKE, 16, None) == 6
+    assert lib.readout_blend(None, 1, FAKE, FAKE, 1, 10, 0.35, None) == 1
+    assert lib.readout_blend(FAKE, 1, FAKE, FAKE, 1, 0, 0.35, None) == 2
+    assert lib.readout_blend(FAKE, 1, FAKE + 4, FAKE, 1, 10, 0.35, None) == 4
+    arr = (mb.CBank * 1)(_bank(ema=FAKE + 0x5000))
+    assert lib.ema_update(arr, 1, 1.0, None) == 5
+    assert lib.ema_update(None, 1, 0.5, None) == 1
+    assert lib.muon_device_status(None, 4096, None, 0) == 1
+    assert lib.muon_set_debug(3, 1.0) == 5
+    assert lib.muon_set_debug(0, 0.0) == 0
