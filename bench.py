@@ -1,0 +1,361 @@
+#!/usr/bin/env python
+"""Benchmark: Muon optimizer steps/s on the GPT-124M matrix bank (B200).
+
+Workload: 48 x 768x768, 12 x 768x3072, 12 x 3072x768 bf16 parameters (84.9 M),
+bf16 gradients N(0, 1e-3^2) plus a rank-4 spike at 10x RMS, fp32 momentum,
+mu = 0.95 Nesterov, five quintic Newton-Schulz steps (3.4445, -4.7750, 2.0315),
+lr 0.05, no weight decay. A step is one muon_step over the whole bank:
+momentum + norm -> 15 Newton-Schulz GEMM launches -> scaled parameter write.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank steps its own
+bank (independent problems, no collective on the data path: weak scaling) and
+rank 0 prints one JSON line with the max-over-ranks device time.
+`--impl reference` times the CPU oracle (host cores) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Muon steps/s on GPT-124M matrix bank; NS TFLOP/s as % bf16 tensor peak"
+UNIT = "steps/s"
+WORKLOAD_ID = 2
+LAUNCHES_PER_STEP_FIXED = 3  # momentum+norm, norm finalize, update
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], burst=p["bf16_tflops"],
+                    sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, burst=1590.0, sustained=1400.0, src="fallback")
+
+
+def _workload():
+    import muon_inputs as mi
+    return mi.workloads()[WORKLOAD_ID]
+
+
+def _ns_flops(w) -> float:
+    """Algorithmic Newton-Schulz flops of one step: per matrix and iteration
+    r(r+1)c (symmetric Gram) + r^2(r+1) (symmetric square) + 2r^2c (B X),
+    r = min(rows, cols), c = max(rows, cols)."""
+    k = len(w.hp["coeffs"])
+    tot = 0.0
+    for b in w.banks:
+        r, c = min(b.rows, b.cols), max(b.rows, b.cols)
+        tot += b.count * k * (r * (r + 1) * c + r * r * (r + 1) + 2.0 * r * r * c)
+    return tot
+
+
+def _config(w, extra=None):
+    c = {"workload": "gpt124m_matrix_bank",
+         "banks": [f"{b.count}x{b.rows}x{b.cols}" for b in w.banks],
+         "params": w.n_params, "param_dtype": w.param_dtype, "grad_dtype": w.grad_dtype,
+         "momentum": "fp32, mu=0.95, nesterov", "ns_steps": len(w.hp["coeffs"]),
+         "coeffs": list(w.hp["coeffs"][0]), "lr": w.hp["lr"], "weight_decay": w.hp["weight_decay"],
+         "grads": "N(0,1e-3^2) + rank-4 spike at 10x RMS",
+         "l2": "inputs larger than L2: ~1.2 GB touched per step (126 MB L2), no flush",
+         "parallelism": "replica per GPU (independent banks)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# --------------------------------------------------------------- CPU oracle
+def _cpu_threads():
+    try:
+        import numpy  # noqa: F401
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def _oracle_sample_time(w, budget_s: float, start_step: int = 0):
+    """Oracle Muon step on matrices of the bank, cycling the three shapes,
+    until budget_s of CPU work; returns (seconds per full-bank step, sample
+    description)."""
+    import numpy as np
+    import muon_inputs as mi
+    import oracle
+    per_shape = {b: [] for b in range(len(w.banks))}
+    t_start = time.perf_counter()
+    idx = 0
+    while True:
+        for b, spec in enumerate(w.banks):
+            i = idx % spec.count
+            th = oracle.as_f64(mi.make_params(w, b, [i])[0])
+            g = oracle.as_f64(mi.make_grads(w, b, start_step, [i])[0])
+            m = np.zeros_like(g)
+            t0 = time.perf_counter()
+            oracle.muon_step(th, g, m, w.hp, w.param_dtype)
+            per_shape[b].append(time.perf_counter() - t0)
+        idx += 1
+        if time.perf_counter() - t_start >= budget_s or idx >= 12:
+            break
+    full = sum(w.banks[b].count * statistics.mean(ts) for b, ts in per_shape.items())
+    n = sum(len(ts) for ts in per_shape.values())
+    desc = (f"oracle muon_step (float64, numpy) on {n} matrices ({idx} of each shape "
+            f"{', '.join(f'{s.rows}x{s.cols}' for s in w.banks)}), mean time per shape "
+            f"scaled by the bank's counts {[s.count for s in w.banks]}")
+    return full, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = _workload()
+    for _ in range(args.warmup):
+        _oracle_sample_time(w, 0.0)
+    times = []
+    desc = ""
+    for s in range(args.steps):
+        t, desc = _oracle_sample_time(w, 0.0, start_step=s)
+        times.append(t)
+    spb = statistics.median(times)
+    v = 1.0 / spb
+    cores = _cpu_threads()
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": spb * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": _config(w),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "each step: " + desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- GPU path
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in open(self.path):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        top = max(sm)
+        loaded = [x for x in sm if x >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+    import muon_inputs as mi
+    import muon_newton_schulz_05_b200 as mb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = _workload()
+    peaks = _peaks()
+
+    # -------- inputs (host-generated, seeded, uploaded before timing)
+    banks, host_grads = [], []
+    for b, spec in enumerate(w.banks):
+        th = mi.make_params(w, b).to(dev)
+        g = mi.make_grads(w, b, 0)
+        host_grads.append(g.pin_memory())
+        banks.append(mb.Bank(th, g.to(dev), torch.zeros(th.shape, dtype=torch.float32, device=dev)))
+    ws = mb.alloc_workspace([bk.shape for bk in banks], device=dev)
+    H = mb.Hparams.from_dict(w.hp)
+    stream = torch.cuda.current_stream(dev)
+    flops_step = _ns_flops(w)
+    k = len(w.hp["coeffs"])
+    launches_per_step = LAUNCHES_PER_STEP_FIXED + 3 * k
+
+    for _ in range(args.warmup):
+        mb.muon_step(banks, H, ws)
+    torch.cuda.synchronize()
+    assert mb.device_status(ws) == 0
+
+    # -------- timed region: K steps, device time, NS chain bracketed live
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * K)]
+    for e in ev:  # materialise the event handles before timing
+        e.record(stream)
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_begin.record(stream)
+    for s in range(K):
+        e_step0, e_ns0, e_ns1, e_step1 = ev[4 * s:4 * s + 4]
+        e_step0.record(stream)
+        mb.set_ns_events(e_ns0, e_ns1)
+        mb.muon_step(banks, H, ws)
+        e_step1.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t_begin.elapsed_time(t_end)
+    ns_ms = [ev[4 * s + 1].elapsed_time(ev[4 * s + 2]) for s in range(K)]
+    pre_ms = [ev[4 * s].elapsed_time(ev[4 * s + 1]) for s in range(K)]
+    post_ms = [ev[4 * s + 2].elapsed_time(ev[4 * s + 3]) for s in range(K)]
+    assert mb.device_status(ws) == 0
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = world * K / (total_ms / 1e3)
+
+    ns_avg_ms = statistics.mean(ns_ms)
+    achieved = flops_step / (ns_avg_ms * 1e-3) / 1e12
+    elem_bytes = sum(b.count * b.rows * b.cols for b in w.banks)
+    # algorithmic bytes of the two elementwise passes per element:
+    # momentum+norm: G bf16 read 2, M read+write 8, iterate hi+lo write 4 = 14
+    # update: iterate hi+lo read 4, theta bf16 read+write 4 = 8
+    pre_gbs = elem_bytes * 14 / (statistics.mean(pre_ms) * 1e-3) / 1e9
+    post_gbs = elem_bytes * 8 / (statistics.mean(post_ms) * 1e-3) / 1e9
+
+    # -------- end to end through the public API with host buffers
+    e2e = None
+    if rank == 0 or world > 1:
+        host_params = [torch.empty(bk.param.shape, dtype=bk.param.dtype).pin_memory() for bk in banks]
+        h2d = sum(g.numel() * g.element_size() for g in host_grads)
+        d2h = sum(p.numel() * p.element_size() for p in host_params)
+        E = args.e2e_steps
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(E):
+            for bk, g in zip(banks, host_grads):
+                bk.grad.copy_(g, non_blocking=True)
+            mb.muon_step(banks, H, ws)
+            for bk, hp_ in zip(banks, host_params):
+                hp_.copy_(bk.param, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "what": "per step: pinned host->device copy of the bf16 gradients, muon_step, "
+                       "device->host copy of the updated bf16 parameters"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        spb, desc = _oracle_sample_time(w, 15.0)
+        cpu = {"value": 1.0 / spb, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+               "sample": desc}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak = peaks["sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(w),
+        "roofline": {
+            "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None,
+            "kernel": "ns_gemm_kernel (the 15 launches of one Newton-Schulz chain)",
+            "flops_per_launch": flops_step, "launch_ms": ns_avg_ms,
+            "peak_kind": f"bf16 dense sustained, {peaks['src']}",
+            "frac_of_burst": achieved / peaks["burst"],
+        },
+        "breakdown_ms": {"momentum_norm": statistics.mean(pre_ms), "ns_chain": ns_avg_ms,
+                         "update": statistics.mean(post_ms)},
+        "elementwise_gbs": {"momentum_norm": pre_gbs, "update": post_gbs, "peak": peaks["hbm"]},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

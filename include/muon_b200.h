@@ -150,6 +150,13 @@ muon_status readout_blend(const void* theta, int32_t theta_dtype, const float* e
  * call blocks the host and is not meant for the hot loop. */
 muon_status muon_device_status(void* ws, size_t ws_bytes, void* stream, int32_t clear);
 
+/* Instrumentation hook, process-wide. The next muon_step, anvil_step or
+ * muon_orthogonalize call records `before_ns` on its stream right before its
+ * first Newton-Schulz launch and `after_ns` right after its last one, then
+ * forgets both. Both are cudaEvent_t handles passed as void* (created by the
+ * caller with timing enabled); NULL, NULL clears a pending pair. */
+muon_status muon_set_ns_events(void* before_ns, void* after_ns);
+
 /* Test hook, process-wide. wait_limit_seconds bounds every device-side wait
  * (default 2 s; values <= 0 restore the default). fault_mode 0 = normal;
  * 1 = the Newton-Schulz kernel's producer withholds the first operand stage of

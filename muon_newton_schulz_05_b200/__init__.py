@@ -4,7 +4,7 @@ Argument marshalling only: every step of the optimizer runs in the library's
 CUDA kernels. PyTorch provides device memory and streams; the C ABI takes raw
 pointers (``tensor.data_ptr()``) and a ``cudaStream_t`` (the current torch
 stream unless one is given). Importing this module fails if the compiled
-library is missing; build it with ``python -m muon_newton_schulz_05_b200.build``.
+library is missing; build it with ``python muon_newton_schulz_05_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmuonb200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m muon_newton_schulz_05_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python muon_newton_schulz_05_b200/build.py` "
         "(this package has no fallback implementation)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -35,7 +35,7 @@ STATUS_NAMES = {
 
 EXPORTED = ("muon_abi_version", "muon_status_string", "muon_workspace_size", "muon_step",
             "anvil_step", "muon_orthogonalize", "ema_update", "readout_blend",
-            "muon_device_status", "muon_set_debug")
+            "muon_device_status", "muon_set_debug", "muon_set_ns_events")
 
 
 class MuonError(RuntimeError):
@@ -73,6 +73,7 @@ _sig = {
     "readout_blend": (_i32, [_vp, _i32, _vp, _vp, _i32, _i64, _f, _vp]),
     "muon_device_status": (_i32, [_vp, _sz, _vp, _i32]),
     "muon_set_debug": (_i32, [_i32, ctypes.c_double]),
+    "muon_set_ns_events": (_i32, [_vp, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)
@@ -252,6 +253,14 @@ def set_debug(fault_mode: int = 0, wait_limit_seconds: float = 0.0) -> None:
     _check(_lib.muon_set_debug(fault_mode, wait_limit_seconds), "muon_set_debug")
 
 
+def set_ns_events(before, after) -> None:
+    """The next step call records these torch.cuda.Events around its
+    Newton-Schulz launches (instrumentation for the benchmark)."""
+    _check(_lib.muon_set_ns_events(before.cuda_event if before is not None else None,
+                                   after.cuda_event if after is not None else None),
+           "muon_set_ns_events")
+
+
 def raw_library():
     """The ctypes handle (used by tests that call the C ABI directly)."""
     return _lib
@@ -263,5 +272,5 @@ def loaded_library_path() -> str:
 
 __all__: List[str] = ["Bank", "Hparams", "MuonError", "workspace_size", "alloc_workspace",
                       "muon_step", "anvil_step", "orthogonalize", "ema_update", "readout_blend",
-                      "device_status", "set_debug", "status_string", "abi_version",
+                      "device_status", "set_debug", "set_ns_events", "status_string", "abi_version",
                       "raw_library", "CBank", "CHparams", "EXPORTED", "F32", "BF16"]

@@ -1,6 +1,8 @@
 """Build libmuonb200.so in-tree with nvcc for sm_100a.
 
-Usage: python -m muon_newton_schulz_05_b200.build [--verbose-ptxas]
+Usage: python muon_newton_schulz_05_b200/build.py [--verbose-ptxas]
+(run by path: the script does not import the package, so it works before
+the library exists)
 The CUDA runtime is linked statically; the driver entry point used for TMA
 descriptors is looked up at run time, so the library has no -lcuda dependency.
 """

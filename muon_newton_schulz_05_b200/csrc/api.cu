@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "muon_b200.h"
 #include "plan.cuh"
@@ -23,6 +24,7 @@ struct DebugState {
 DebugState g_debug;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+cudaEvent_t g_ev_before = nullptr, g_ev_after = nullptr;
 std::mutex g_mu;
 
 struct DeviceState {
@@ -251,6 +253,13 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
     gp.bank[b] = plans[b];
     if ((st = encode_bank_maps(plans[b], gp.maps[b])) != MUON_OK) return st;
   }
+  cudaEvent_t ev_before = nullptr, ev_after = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    std::swap(ev_before, g_ev_before);
+    std::swap(ev_after, g_ev_after);
+  }
+  if (ev_before && cudaEventRecord(ev_before, stream) != cudaSuccess) return MUON_ERR_CUDA;
   for (int it = 0; it < hp->ns_steps; ++it) {
     gp.iter = it;
     gp.cur = it & 1;
@@ -269,6 +278,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
       if (launch_ns_gemm(gp, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
     }
   }
+  if (ev_after && cudaEventRecord(ev_after, stream) != cudaSuccess) return MUON_ERR_CUDA;
 
   // ---- scale, decay, parameter write (+ EMA), or O out
   UpdParams up;
@@ -444,6 +454,14 @@ muon_status muon_device_status(void* ws, size_t ws_bytes, void* stream, int32_t 
     if (cudaStreamSynchronize(s) != cudaSuccess) return MUON_ERR_CUDA;
   }
   return v == 0 ? MUON_OK : static_cast<muon_status>(v);
+}
+
+muon_status muon_set_ns_events(void* before_ns, void* after_ns) {
+  if ((before_ns == nullptr) != (after_ns == nullptr)) return MUON_ERR_NULL;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_ev_before = static_cast<cudaEvent_t>(before_ns);
+  g_ev_after = static_cast<cudaEvent_t>(after_ns);
+  return MUON_OK;
 }
 
 muon_status muon_set_debug(int32_t fault_mode, double wait_limit_seconds) {
