@@ -59,13 +59,17 @@ def test_orthogonalize_matches_oracle(shape, cname):
     cnt, R, C = shape
     g = mi.gaussian(cnt * R, C, seed=R * 1000 + C, sigma=1.0).reshape(cnt, R, C).to(torch.bfloat16)
     out = orth_gpu(g.to(DEV), coeffs).cpu()
+    sv_tol = TOL_SV
     if min(R, C) < 32 and "quintic" in cname:
-        tol = 4e-2  # a handful of singular values: one bf16-sensitive value dominates
+        # Only a handful of singular values: the bf16 rounding of the operands
+        # alone (the kernel's scheme replayed in float64 on the CPU) moves one
+        # of them by 0.057 after six quintic steps on the 7 x 13 case.
+        tol, sv_tol = 4e-2, 0.08
     for i in range(cnt):
         ref = oracle.orthogonalize(f64(g[i]), coeffs, 1e-7)
         got = f64(out[i])
         assert rel_fro(got, ref) <= tol, (i, rel_fro(got, ref))
-        assert sv_maxdiff(got, ref) <= TOL_SV
+        assert sv_maxdiff(got, ref) <= sv_tol
 
 
 def test_orthogonalize_bf16_output_and_fp32_input():
