@@ -7,6 +7,17 @@ TOL_UPDATE = 2e-2      # orthogonalised update, relative Frobenius
 TOL_SV = 0.05          # every output singular value, absolute
 
 
+def update_tols(rows, cols):
+    """(relative Frobenius, singular-value) tolerances of the orthogonalised
+    update. With fewer than 32 singular values one bf16-sensitive value
+    dominates: replaying the kernel's own bf16 rounding scheme in float64 on
+    the CPU gives up to 3.3e-2 / 0.057 on 7 x 13 and 2.1e-2 on 8 x 1, so tiny
+    matrices get 4e-2 / 0.08."""
+    if min(rows, cols) < 32:
+        return 4e-2, 0.08
+    return TOL_UPDATE, TOL_SV
+
+
 def rel_fro(got, ref):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

@@ -14,7 +14,7 @@ import torch
 import muon_inputs as mi
 import oracle
 from _parity import (TOL_BUFFER, TOL_SV, TOL_UPDATE, buffer_ok, delta_ok, rel_fro,
-                     sv_maxdiff)
+                     bf16_ulp, sv_maxdiff, update_tols)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,10 +61,7 @@ def test_orthogonalize_matches_oracle(shape, cname):
     out = orth_gpu(g.to(DEV), coeffs).cpu()
     sv_tol = TOL_SV
     if min(R, C) < 32 and "quintic" in cname:
-        # Only a handful of singular values: the bf16 rounding of the operands
-        # alone (the kernel's scheme replayed in float64 on the CPU) moves one
-        # of them by 0.057 after six quintic steps on the 7 x 13 case.
-        tol, sv_tol = 4e-2, 0.08
+        tol, sv_tol = update_tols(R, C)
     for i in range(cnt):
         ref = oracle.orthogonalize(f64(g[i]), coeffs, 1e-7)
         got = f64(out[i])
@@ -122,18 +119,19 @@ def _muon_run(w, steps, check_steps, sample, hp_override=None):
             assert ok, ("momentum", b, step, r)
             R, C = bk.shape[1:]
             s = oracle.shape_scale(R, C)
+            tol_o, tol_sv = update_tols(R, C)
             for i in sample(b, bk.shape[0]):
                 U = oracle.nesterov_lookahead(Mref[i], f64(G[i]), hp["mu"], bool(hp["nesterov"]))
                 O = oracle.orthogonalize(U, hp["coeffs"], hp["eps"])
                 # the NS path on the GPU's own U
                 Ug = torch.from_numpy(U.astype(np.float32))[None].to(DEV)
                 Og = f64(orth_gpu(Ug, hp["coeffs"])[0])
-                assert rel_fro(Og, O) <= TOL_UPDATE, ("O", b, i, step, rel_fro(Og, O))
-                assert sv_maxdiff(Og, O) <= TOL_SV
+                assert rel_fro(Og, O) <= tol_o, ("O", b, i, step, rel_fro(Og, O))
+                assert sv_maxdiff(Og, O) <= tol_sv
                 # parameter step (teacher-forced on the GPU's theta_old)
                 t0 = f64(th0[i])
                 dref = oracle.decoupled_update(t0, O, hp["lr"], hp["weight_decay"], s) - t0
-                ok, r = delta_ok(t0, f64(bk.param[i]), dref, w.param_dtype)
+                ok, r = delta_ok(t0, f64(bk.param[i]), dref, w.param_dtype, tol_o)
                 assert ok, ("delta", b, i, step, r)
     return banks
 
@@ -232,8 +230,11 @@ def test_anvil_mask_decisions_agree_where_unambiguous():
     mask = oracle.cautious_mask(O, Ms)
     t0 = f64(th[0])
     lr, wd, s = 0.05, 0.5, 1.0
-    # recover the GPU's decay decision: theta_new = t0 - lr wd m t0 - lr s O
-    Og = f64(orth_gpu(torch.from_numpy(Mf.astype(np.float32))[None].to(DEV), hp["coeffs"])[0])
+    # recover the GPU's decay decision: theta_new = t0 - lr wd m t0 - lr s O.
+    # O must be the step's own: the orthogonalisation of the GPU's fast momentum
+    # reproduces it bit for bit, while an input one fp32 ulp away re-draws the
+    # ~1 % bf16 rounding error (elementwise up to ~8 % of rms(O) in the tails).
+    Og = f64(orth_gpu(bank.momentum.clone(), hp["coeffs"])[0])
     pred_nodecay = t0 - lr * s * Og
     pred_decay = t0 - lr * wd * t0 - lr * s * Og
     got = f64(bank.param[0])
@@ -241,9 +242,13 @@ def test_anvil_mask_decisions_agree_where_unambiguous():
     # O carries ~1 % relative error; its sign is certain where |O| is well
     # above that, and M_slow is fp32-exact against the oracle
     rms = lambda a: np.sqrt(np.mean(a * a))
-    sure = (np.abs(O) > 0.2 * rms(O)) & (np.abs(Ms) > 1e-3 * rms(Ms)) & (np.abs(t0) > 1e-4)
-    assert sure.sum() > 0.5 * sure.size
-    assert np.array_equal(decided[sure], mask[sure])
+    sure = (np.abs(O) > 0.2 * rms(O)) & (np.abs(Ms) > 1e-3 * rms(Ms))
+    # the decision is recoverable only where the decay term is well above the
+    # bf16 rounding of the stored parameter
+    sure &= lr * wd * np.abs(t0) > 3.0 * bf16_ulp(got)
+    assert sure.sum() > 0.3 * sure.size, sure.sum()
+    bad = int(np.sum(decided[sure] != mask[sure]))
+    assert bad == 0, (bad, int(sure.sum()))
 
 
 def test_standalone_ema_update():
