@@ -132,6 +132,32 @@ muon_status muon_orthogonalize(const void* in, int32_t in_dtype, void* out, int3
                                int64_t count, int64_t rows, int64_t cols,
                                const muon_hparams* hp, void* ws, size_t ws_bytes, void* stream);
 
+/* muon_orthogonalize without a caller workspace. The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory themselves, for example a plug-in inside a host application
+ * that owns every device allocation, or a latency-critical loop where a
+ * cudaMalloc (which may synchronise the whole device) is not allowed. Its
+ * scratch memory is one array of MUON_STATIC_SCRATCH_BYTES in the library's
+ * own device memory, reserved on every GPU that loads the library until the
+ * process exits. Arguments and results are those of muon_orthogonalize
+ * (inputs and outputs still belong to the caller).
+ *   - A bank whose muon_workspace_size exceeds MUON_STATIC_SCRATCH_BYTES is
+ *     rejected with MUON_ERR_WORKSPACE before anything is launched (32 MiB
+ *     holds e.g. one 768 x 3072 or two 1024 x 1024 matrices).
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     each call clears the part that must start at zero. Calls whose work
+ *     overlaps on the GPU (other streams, other host threads) race on it.
+ *   - The device status word used by bounded waits lives in the array too and
+ *     is cleared at the start of every call, so a timeout here is not visible
+ *     to muon_device_status; use muon_orthogonalize to observe it.
+ * Calls no cudaMalloc, cudaFree or other allocating routine. */
+#define MUON_STATIC_SCRATCH_BYTES (32u << 20)
+muon_status muon_orthogonalize_static(const void* in, int32_t in_dtype, void* out,
+                                      int32_t out_dtype, int64_t count, int64_t rows,
+                                      int64_t cols, const muon_hparams* hp, void* stream);
+
 /* EMA of the parameters ("ANVIL II와 가중치 평균", averaging equation):
  * ema <- beta ema + (1 - beta) param, for every bank with ema != NULL.
  * 0 <= beta < 1. Banks whose ema is NULL are skipped. */

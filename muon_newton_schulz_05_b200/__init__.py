@@ -35,7 +35,8 @@ STATUS_NAMES = {
 
 EXPORTED = ("muon_abi_version", "muon_status_string", "muon_workspace_size", "muon_step",
             "anvil_step", "muon_orthogonalize", "ema_update", "readout_blend",
-            "muon_device_status", "muon_set_debug", "muon_set_ns_events")
+            "muon_device_status", "muon_set_debug", "muon_set_ns_events",
+            "muon_orthogonalize_static")
 
 
 class MuonError(RuntimeError):
@@ -74,6 +75,8 @@ _sig = {
     "muon_device_status": (_i32, [_vp, _sz, _vp, _i32]),
     "muon_set_debug": (_i32, [_i32, ctypes.c_double]),
     "muon_set_ns_events": (_i32, [_vp, _vp]),
+    "muon_orthogonalize_static": (_i32, [_vp, _i32, _vp, _i32, _i64, _i64, _i64,
+                                         ctypes.POINTER(CHparams), _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)

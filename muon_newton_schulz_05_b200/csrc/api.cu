@@ -456,6 +456,62 @@ muon_status muon_device_status(void* ws, size_t ws_bytes, void* stream, int32_t 
   return v == 0 ? MUON_OK : static_cast<muon_status>(v);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------- fixed scratch, no allocation
+// Scratch for muon_orthogonalize_static: one file-scope device array. Host code
+// must not use its name as a device address; the address is looked up once per
+// device with cudaGetSymbolAddress, with that device current.
+static __device__ __align__(256) unsigned char g_static_scratch[MUON_STATIC_SCRATCH_BYTES];
+
+namespace {
+void* g_static_ptr[64] = {};
+
+muon_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MUON_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+      return MUON_ERR_CUDA;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return MUON_OK;
+}
+}  // namespace
+
+extern "C" {
+
+muon_status muon_orthogonalize_static(const void* in, int32_t in_dtype, void* out,
+                                      int32_t out_dtype, int64_t count, int64_t rows,
+                                      int64_t cols, const muon_hparams* hp, void* stream) {
+  if (!in || !out || !hp) return MUON_ERR_NULL;
+  muon_status st = check_shape(count, rows, cols);
+  if (st != MUON_OK) return st;
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return MUON_ERR_DTYPE;
+  if (!aligned16(in) || !aligned16(out)) return MUON_ERR_ALIGN;
+  if ((st = check_ns(hp)) != MUON_OK) return st;
+  muon_bank bank;
+  std::memset(&bank, 0, sizeof(bank));
+  bank.count = count;
+  bank.rows = rows;
+  bank.cols = cols;
+  const size_t need = muon_workspace_size(&bank, 1);
+  if (need == 0 || need > MUON_STATIC_SCRATCH_BYTES) return MUON_ERR_WORKSPACE;
+  const size_t n = static_cast<size_t>(count * rows * cols);
+  if (overlap(in, n * (in_dtype == MUON_BF16 ? 2 : 4), out, n * (out_dtype == MUON_BF16 ? 2 : 4)))
+    return MUON_ERR_ALIAS;
+  void* ws = nullptr;
+  if ((st = static_scratch(&ws)) != MUON_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the status word is the only part of the scratch that must start at zero
+  if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return MUON_ERR_CUDA;
+  OrthoIO io{in, in_dtype, out, out_dtype};
+  return run_step(Variant::kOrtho, &bank, 1, hp, ws, MUON_STATIC_SCRATCH_BYTES, s, &io);
+}
+
 muon_status muon_set_ns_events(void* before_ns, void* after_ns) {
   if ((before_ns == nullptr) != (after_ns == nullptr)) return MUON_ERR_NULL;
   std::lock_guard<std::mutex> lk(g_mu);
