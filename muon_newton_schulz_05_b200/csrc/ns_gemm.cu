@@ -7,13 +7,14 @@
 // ("Muonとは" / "Muonが登場": approximate orthogonalisation by Newton-Schulz
 // iteration, bf16 operands; the polynomial step is the method statement's).
 //
-// Block layout (192 threads, one block per SM):
+// Block layout (320 threads, one block per SM):
 //   warp 0     one thread issues TMA loads into a 4-stage smem ring
 //   warp 1     allocates 512 TMEM columns; one thread issues tcgen05.mma
 //              (M=128, N=256, K=16, bf16 in, fp32 accumulate) into one of two
 //              256-column accumulators
-//   warps 2..5 epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
-//              32*(w%4)..+31, i.e. tile rows), apply the phase's axpy and store
+//   warps 2..9 epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
+//              32*(w%4)..+31, i.e. tile rows; two warps per lane quadrant split
+//              the 256 columns), apply the phase's axpy and store
 // Tiles are 128 x 256 with K in 64-element (128-byte, swizzled) steps. The
 // epilogue of tile t overlaps the MMAs of tile t+1 through the two
 // accumulators. Every wait is bounded (muon::mbar_wait).
@@ -117,10 +118,37 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_majo
 }
 
 // ---------------------------------------------------------------- epilogues
-// Gram / Poly: row `row` of the tile, columns col0 .. col0+31 in v[]. Stores
-// the upper part (col >= row) in place and mirrors the strict upper part.
+// Each epilogue thread owns one accumulator row and handles 64 columns at a
+// time: its global inputs (the previous iterate for Apply, A for Poly) are
+// loaded first, then two 32-column TMEM loads share one wait.
+struct EpiIn {
+  uint4 x[8];  // Apply: hi of 64 columns; Poly: A of 64 columns
+  uint4 y[8];  // Apply: lo of 64 columns
+};
+
+__device__ __forceinline__ void epi_prefetch(const NsGemmParams& p, const BankPlan& bp, int mat,
+                                             int row, int col0, EpiIn& in) {
+  if (p.phase == kApply) {
+    const size_t off = static_cast<size_t>(mat) * bp.Rp * bp.Cp + static_cast<size_t>(row) * bp.Cp + col0;
+    const uint4* hin = reinterpret_cast<const uint4*>(bp.hi[p.cur] + off);
+    const uint4* lio = reinterpret_cast<const uint4*>(bp.lo + off);
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      in.x[g] = hin[g];
+      in.y[g] = lio[g];
+    }
+  } else if (p.phase == kPoly && col0 + 63 >= row) {
+    const size_t rp = static_cast<size_t>(bp.rp);
+    const uint4* ain = reinterpret_cast<const uint4*>(bp.A + static_cast<size_t>(mat) * rp * rp + row * rp + col0);
+#pragma unroll
+    for (int g = 0; g < 8; ++g) in.x[g] = ain[g];
+  }
+}
+
+// Gram / Poly: columns col0 .. col0+31 of row `row` in v[]; a4 = A there (Poly).
+// Stores the upper part (col >= row) in place and mirrors the strict upper part.
 __device__ __forceinline__ void epilogue_sym(const NsGemmParams& p, const BankPlan& bp, int mat,
-                                             int row, int col0, float (&v)[32]) {
+                                             int row, int col0, float (&v)[32], const uint4* a4) {
   if (col0 + 31 < row) return;  // entirely below the diagonal: the mirror covers it
   const size_t rp = static_cast<size_t>(bp.rp);
   const size_t mbase = static_cast<size_t>(mat) * rp * rp;
@@ -133,11 +161,9 @@ __device__ __forceinline__ void epilogue_sym(const NsGemmParams& p, const BankPl
       for (int t = 0; t < 32; ++t) v[t] *= s2;
     }
   } else {
-    const uint4* ain = reinterpret_cast<const uint4*>(bp.A + mbase + row * rp + col0);
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      const uint4 w = ain[g];
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      const uint32_t ww[4] = {a4[g].x, a4[g].y, a4[g].z, a4[g].w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         v[8 * g + 2 * h] = fmaf(p.c, v[8 * g + 2 * h], p.b * bf16_lo_f(ww[h]));
@@ -166,11 +192,12 @@ __device__ __forceinline__ void epilogue_sym(const NsGemmParams& p, const BankPl
     if (col0 + t > row) ocol[static_cast<size_t>(t) * rp] = ps[t];
 }
 
-// Apply: x' = alpha x + beta D with x = hi + lo; writes hi' (other buffer) and lo.
+// Apply: x' = alpha x + beta D with x = hi + lo (h4, l4: 32 columns);
+// writes hi' (other buffer) and lo.
 __device__ __forceinline__ void epilogue_apply(const NsGemmParams& p, const BankPlan& bp, int mat,
-                                               int row, int col0, const float (&v)[32]) {
+                                               int row, int col0, const float (&v)[32],
+                                               const uint4* h4, const uint4* l4) {
   const size_t off = static_cast<size_t>(mat) * bp.Rp * bp.Cp + static_cast<size_t>(row) * bp.Cp + col0;
-  const uint4* hin = reinterpret_cast<const uint4*>(bp.hi[p.cur] + off);
   uint4* hout = reinterpret_cast<uint4*>(bp.hi[p.cur ^ 1] + off);
   uint4* lio = reinterpret_cast<uint4*>(bp.lo + off);
   float alpha = p.a, beta = 1.0f;
@@ -181,10 +208,8 @@ __device__ __forceinline__ void epilogue_apply(const NsGemmParams& p, const Bank
   }
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
-    const uint4 h4 = hin[g];
-    const uint4 l4 = lio[g];
-    const uint32_t hw[4] = {h4.x, h4.y, h4.z, h4.w};
-    const uint32_t lw[4] = {l4.x, l4.y, l4.z, l4.w};
+    const uint32_t hw[4] = {h4[g].x, h4[g].y, h4[g].z, h4[g].w};
+    const uint32_t lw[4] = {l4[g].x, l4[g].y, l4[g].z, l4[g].w};
     uint32_t ho[4], lo[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
@@ -198,6 +223,18 @@ __device__ __forceinline__ void epilogue_apply(const NsGemmParams& p, const Bank
     hout[g] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
     lio[g] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
+}
+
+__device__ __forceinline__ void epilogue_chunk(const NsGemmParams& p, const BankPlan& bp, int mat,
+                                               int row, int col0, const uint32_t (&r)[32],
+                                               const EpiIn& in, int part) {
+  float v[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+  if (p.phase == kApply)
+    epilogue_apply(p, bp, mat, row, col0, v, in.x + 4 * part, in.y + 4 * part);
+  else
+    epilogue_sym(p, bp, mat, row, col0, v, in.x + 4 * part);
 }
 
 // Waits that ignore the abort flag, used only to drain in-flight work.
@@ -232,7 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], kEpiWarps);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -320,29 +357,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     }
   } else {
     // ---------------------------------------------------------------- epilogue
+    // warp w may read TMEM lanes 32*(w%4)..+31 (tile rows); warps 2..5 take
+    // accumulator columns 0..127 and warps 6..9 columns 128..255.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.tile_begin[p.nbanks]; tile += gridDim.x) {
       const Tile T = decode_tile(p, tile);
+      const BankPlan& bp = p.bank[T.bank];
+      const int row = T.m0 + 32 * q + lane;
+      EpiIn in;
+      epi_prefetch(p, bp, T.mat, row, T.n0 + half * 128, in);
       // the tcgen05.ld below is warp-collective: leave only if the whole warp does
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, limit);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const BankPlan& bp = p.bank[T.bank];
-      const int row = T.m0 + 32 * q + lane;
-      const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * kBN);
-      for (int j = 0; j < kBN / 32; ++j) {
-        uint32_t r[32];
-        tmem_ld32(tb + 32 * j, r);
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                          static_cast<uint32_t>(acc * kBN + half * 128);
+#pragma unroll 1
+      for (int jj = 0; jj < 2; ++jj) {
+        const int col0 = T.n0 + half * 128 + jj * 64;
+        if (jj > 0) epi_prefetch(p, bp, T.mat, row, col0, in);
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tb + jj * 64, r0);
+        tmem_ld32(tb + jj * 64 + 32, r1);
         tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
-        if (p.phase == kApply)
-          epilogue_apply(p, bp, T.mat, row, T.n0 + 32 * j, v);
-        else
-          epilogue_sym(p, bp, T.mat, row, T.n0 + 32 * j, v);
+        epilogue_chunk(p, bp, T.mat, row, col0, r0, in, 0);
+        epilogue_chunk(p, bp, T.mat, row, col0 + 32, r1, in, 1);
       }
       tc_fence_before();
       __syncwarp();

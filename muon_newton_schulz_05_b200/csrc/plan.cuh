@@ -26,7 +26,8 @@ constexpr int kATileBytes = kBM * kBK * 2;
 constexpr int kBTileBytes = kBN * kBK * 2;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 + 256;
-constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kEpiWarps = 8;      // two per TMEM lane quadrant
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, then epilogue
 constexpr int kChunk = 8192;       // padded elements per block in the momentum pass
 constexpr int kMaxMaps = 6;
 
