@@ -72,7 +72,7 @@ muon_status check_shape(int64_t count, int64_t rows, int64_t cols) {
   // TMA coordinates and tile indices are 32-bit
   if (count * Rp >= (int64_t(1) << 31) || count * rp >= (int64_t(1) << 31)) return MUON_ERR_SHAPE;
   if (Rp >= (int64_t(1) << 24) || Cp >= (int64_t(1) << 24)) return MUON_ERR_SHAPE;
-  const int64_t tiles = count * (Rp / kBM) * (Cp / kBN);
+  const int64_t tiles = count * (Rp / kTile) * (Cp / kTile);
   const int64_t chunks = (Rp * Cp + kChunk - 1) / kChunk;
   if (tiles >= (int64_t(1) << 30) || count * chunks >= (int64_t(1) << 30)) return MUON_ERR_SHAPE;
   return MUON_OK;
@@ -146,9 +146,9 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
     p.rp = p.tall ? p.Cp : p.Rp;
     const size_t padded = static_cast<size_t>(p.Rp) * p.Cp;
     p.chunks = static_cast<int>((padded + kChunk - 1) / kChunk);
-    const int nb = p.rp / kBN;
-    p.tiles_sym = nb * (nb + 1);
-    p.tiles_apply = (p.Rp / kBM) * (p.Cp / kBN);
+    const int nb = p.rp / kTile;
+    p.tiles_sym = nb * (nb + 1) / 2;
+    p.tiles_apply = (p.Rp / kTile) * (p.Cp / kTile);
     const size_t it_bytes = static_cast<size_t>(p.count) * padded * 2;
     const size_t sq_bytes = static_cast<size_t>(p.count) * p.rp * p.rp * 2;
     const size_t o_hi0 = take(it_bytes), o_hi1 = take(it_bytes), o_lo = take(it_bytes);
@@ -274,8 +274,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
         tiles += plans[b].count * (ph == kApply ? plans[b].tiles_apply : plans[b].tiles_sym);
       }
       gp.tile_begin[nbanks] = tiles;
-      const int grid = tiles < sms ? tiles : sms;
-      if (launch_ns_gemm(gp, grid, stream) != cudaSuccess) return MUON_ERR_CUDA;
+      if (launch_ns_gemm(gp, sms, stream) != cudaSuccess) return MUON_ERR_CUDA;
     }
   }
   if (ev_after && cudaEventRecord(ev_after, stream) != cudaSuccess) return MUON_ERR_CUDA;

@@ -7,17 +7,22 @@
 // ("Muonとは" / "Muonが登場": approximate orthogonalisation by Newton-Schulz
 // iteration, bf16 operands; the polynomial step is the method statement's).
 //
-// Block layout (320 threads, one block per SM):
-//   warp 0     one thread issues TMA loads into a 4-stage smem ring
-//   warp 1     allocates 512 TMEM columns; one thread issues tcgen05.mma
-//              (M=128, N=256, K=16, bf16 in, fp32 accumulate) into one of two
-//              256-column accumulators
-//   warps 2..9 epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
-//              32*(w%4)..+31, i.e. tile rows; two warps per lane quadrant split
-//              the 256 columns), apply the phase's axpy and store
-// Tiles are 128 x 256 with K in 64-element (128-byte, swizzled) steps. The
-// epilogue of tile t overlaps the MMAs of tile t+1 through the two
-// accumulators. Every wait is bounded (muon::mbar_wait).
+// CTA pairs (clusters of 2 on one TPC) compute 256 x 256 output tiles with the
+// 2-SM MMA (tcgen05.mma.cta_group::2, M = 256, N = 256, K = 16): each CTA
+// stages its own 128 rows of the A operand and its half (128 rows) of the B
+// operand, so every SM reads 32 KB per 64-deep K step instead of 48 KB.
+// No TMA multicast is used; only the MMA commits arrive on both CTAs.
+//
+// Block layout (320 threads, one block per SM), in both CTAs of a pair:
+//   warp 0     one thread issues this CTA's TMA loads into a 6-stage ring;
+//              completion is counted on the even (leader) CTA's barrier
+//   warp 1     allocates 512 TMEM columns (pair allocation); in the leader one
+//              thread issues the MMAs into one of two 256-column accumulators
+//   warps 2..9 epilogue: tcgen05.ld this CTA's 128 accumulator rows (warp w
+//              reads TMEM lanes 32*(w%4)..+31; two warps per lane quadrant
+//              split the 256 columns), apply the phase's axpy and store
+// The epilogue of tile t overlaps the MMAs of tile t+1 through the two
+// accumulators. Every wait is bounded (muon::mbar_wait*).
 #include <cuda_runtime.h>
 
 #include "plan.cuh"
@@ -31,19 +36,16 @@ struct Tile {
   int b_map, b_mn, b_base;
 };
 
-// Upper tiles of a symmetric product with 2*nb row blocks (128) and nb column
-// blocks (256): row blocks 2p and 2p+1 hold column blocks p .. nb-1.
+// Upper 256 x 256 tiles (diagonal included) of a symmetric product with nb
+// block rows: block row i holds block columns i .. nb-1.
 __device__ __forceinline__ void sym_tile(int t, int nb, int& i, int& j) {
-  int p = 0;
-  for (;;) {
-    const int cnt = 2 * (nb - p);
-    if (t < cnt) break;
-    t -= cnt;
-    ++p;
+  int ii = 0;
+  while (t >= nb - ii) {
+    t -= nb - ii;
+    ++ii;
   }
-  const int per = nb - p;
-  i = 2 * p + t / per;
-  j = p + t % per;
+  i = ii;
+  j = ii + t;
 }
 
 __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
@@ -56,16 +58,16 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   if (p.phase == kApply) {
     T.mat = local / bp.tiles_apply;
     const int t = local - T.mat * bp.tiles_apply;
-    const int nbn = bp.Cp / kBN;
-    T.m0 = (t / nbn) * kBM;
-    T.n0 = (t % nbn) * kBN;
+    const int nbn = bp.Cp / kTile;
+    T.m0 = (t / nbn) * kTile;
+    T.n0 = (t % nbn) * kTile;
   } else {
     T.mat = local / bp.tiles_sym;
     const int t = local - T.mat * bp.tiles_sym;
     int i, j;
-    sym_tile(t, bp.rp / kBN, i, j);
-    T.m0 = i * kBM;
-    T.n0 = j * kBN;
+    sym_tile(t, bp.rp / kTile, i, j);
+    T.m0 = i * kTile;
+    T.n0 = j * kTile;
   }
   const int cur = p.cur;
   const int xbase = T.mat * bp.Rp;   // first row of this matrix in the iterate maps
@@ -98,17 +100,17 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   return T;
 }
 
-// One operand tile of `rows` (MN extent) x 64 (K) into dst.
-//  K-major : boxes of 128 rows x 64 K (16 KB), stacked along MN.
-//  MN-major: boxes of 64 K rows x 64 MN (8 KB), stacked along MN.
-__device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
-                                             int mn_major, int rows, int base, int mn0, int k0) {
+// This CTA's 128 (MN) x 64 (K) slice of an operand tile into dst; completion
+// is counted on the pair leader's barrier bar (shared::cluster address).
+//  K-major : one box of 128 rows x 64 K (16 KB).
+//  MN-major: two boxes of 64 K rows x 64 MN (8 KB each), stacked along MN.
+__device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint32_t bar,
+                                             int mn_major, int base, int mn0, int k0) {
   if (!mn_major) {
-    for (int i = 0; i < rows / 128; ++i)
-      tma_load_2d(dst + i * 16384, map, bar, k0, base + mn0 + 128 * i);
+    tma_load_2d_pair(dst, map, bar, k0, base + mn0);
   } else {
-    for (int j = 0; j < rows / 64; ++j)
-      tma_load_2d(dst + j * 8192, map, bar, mn0 + 64 * j, base + k0);
+    tma_load_2d_pair(dst, map, bar, mn0, base + k0);
+    tma_load_2d_pair(dst + 8192, map, bar, mn0 + 64, base + k0);
   }
 }
 
@@ -246,7 +248,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ NsGemmParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    ns_gemm_kernel(const __grid_constant__ NsGemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
@@ -261,15 +264,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t limit = p.wait_limit_ns;
+  const uint32_t rank = cluster_ctarank();  // 0: pair leader, issues the MMAs
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+  const int ntiles = p.tile_begin[p.nbanks];
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&full[s], 1);   // the leader's: one arrival + both CTAs' bytes
+      mbar_init(&empty[s], 1);  // one multicast commit from the leader's MMAs
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiWarps);
+      mbar_init(&tempty[a], 2 * kEpiWarps);  // the leader's: both CTAs' epilogue warps
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -280,97 +287,114 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       for (int k = 0; k < kMaxMaps; ++k) tma_prefetch_map(&p.maps[b][k]);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // the other CTA's barriers are initialised before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
+      const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
       int stage = 0;
       uint32_t phase = 0;
       int issued_parity[kStages];
       for (int s = 0; s < kStages; ++s) issued_parity[s] = -1;
       bool ok = true;
       bool first = true;
-      for (int tile = blockIdx.x; ok && tile < p.tile_begin[p.nbanks]; tile += gridDim.x) {
+      for (int tile = pair; ok && tile < ntiles; tile += npairs) {
         const Tile T = decode_tile(p, tile);
         const CUtensorMap* amap = &p.maps[T.bank][T.a_map];
         const CUtensorMap* bmap = &p.maps[T.bank][T.b_map];
         for (int kb = 0; kb < T.nkb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, limit)) { ok = false; break; }
+          if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, abort_flag, p.status, limit)) {
+            ok = false;
+            break;
+          }
           const bool withhold = first && p.fault == 1 && blockIdx.x == 0;
           first = false;
           if (!withhold) {
             uint8_t* st = tiles + stage * kStageBytes;
-            mbar_arrive_expect_tx(&full[stage], kStageBytes);
-            load_operand(st, amap, &full[stage], T.a_mn, kBM, T.a_base, T.m0, kb * kBK);
-            load_operand(st + kATileBytes, bmap, &full[stage], T.b_mn, kBN, T.b_base, T.n0, kb * kBK);
+            const uint32_t bar = full_leader + 8u * static_cast<uint32_t>(stage);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+            load_operand(st, amap, bar, T.a_mn, T.a_base, T.m0 + kBM * rank, kb * kBK);
+            load_operand(st + kATileBytes, bmap, bar, T.b_mn, T.b_base, T.n0 + (kBN / 2) * rank,
+                         kb * kBK);
             issued_parity[stage] = static_cast<int>(phase);
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      // make sure no bulk copy is still landing in shared memory
-      for (int s = 0; s < kStages; ++s)
-        if (issued_parity[s] >= 0) drain_wait(&full[s], static_cast<uint32_t>(issued_parity[s]), limit);
+      // the leader's full barriers count both CTAs' bytes: drain them there
+      if (rank == 0)
+        for (int s = 0; s < kStages; ++s)
+          if (issued_parity[s] >= 0) drain_wait(&full[s], static_cast<uint32_t>(issued_parity[s]), limit);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.tile_begin[p.nbanks]; tile += gridDim.x) {
-        const Tile T = decode_tile(p, tile);
-        const uint32_t idesc = idesc_bf16(kBM, kBN, T.a_mn, T.b_mn);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, limit)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-        for (int kb = 0; kb < T.nkb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, limit)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(tiles + stage * kStageBytes);
-          const uint32_t b_addr = a_addr + kATileBytes;
-#pragma unroll
-          for (int ks = 0; ks < kBK / 16; ++ks) {
-            umma_bf16(d_tmem, operand_desc(a_addr, T.a_mn, ks), operand_desc(b_addr, T.b_mn, ks),
-                      idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+      if (rank == 0) {
+        // -------------------------------------------------- MMA issuer (leader)
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int tile = pair; ok && tile < ntiles; tile += npairs) {
+          const Tile T = decode_tile(p, tile);
+          const uint32_t idesc = idesc_bf16(2 * kBM, kBN, T.a_mn, T.b_mn);
+          if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, limit)) {
+            ok = false;
+            break;
           }
-          umma_commit(&empty[stage]);
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+          for (int kb = 0; kb < T.nkb; ++kb) {
+            if (!mbar_wait_cluster(&full[stage], phase, abort_flag, p.status, limit)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(tiles + stage * kStageBytes);
+            const uint32_t b_addr = a_addr + kATileBytes;
+#pragma unroll
+            for (int ks = 0; ks < kBK / 16; ++ks) {
+              umma_bf16_pair(d_tmem, operand_desc(a_addr, T.a_mn, ks),
+                             operand_desc(b_addr, T.b_mn, ks), idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit_pair(&empty[stage]);  // frees this stage in both CTAs
+            if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          }
+          if (!ok) break;
+          umma_commit_pair(&tfull[acc]);
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
         }
-        if (!ok) break;
-        umma_commit(&tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        // every MMA has finished (both CTAs learn it) before TMEM is released
+        umma_commit_pair(done);
       }
-      // every MMA issued by this thread has finished before TMEM is released
-      umma_commit(done);
       drain_wait(done, 0, limit);
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    // warp w may read TMEM lanes 32*(w%4)..+31 (tile rows); warps 2..5 take
-    // accumulator columns 0..127 and warps 6..9 columns 128..255.
+    // warp w may read TMEM lanes 32*(w%4)..+31 (this CTA's tile rows); warps
+    // 2..5 take accumulator columns 0..127 and warps 6..9 columns 128..255.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
+    const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.tile_begin[p.nbanks]; tile += gridDim.x) {
+    for (int tile = pair; tile < ntiles; tile += npairs) {
       const Tile T = decode_tile(p, tile);
       const BankPlan& bp = p.bank[T.bank];
-      const int row = T.m0 + 32 * q + lane;
+      const int row = T.m0 + kBM * static_cast<int>(rank) + 32 * q + lane;
       EpiIn in;
       epi_prefetch(p, bp, T.mat, row, T.n0 + half * 128, in);
       // the tcgen05.ld below is warp-collective: leave only if the whole warp does
-      const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status, limit);
+      const bool got = mbar_wait_cluster(&tfull[acc], acc_phase, abort_flag, p.status, limit);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
@@ -388,7 +412,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -396,10 +420,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // no MMA of the pair and no remote signal is still in flight
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc_pair(tmem_base, 512);
   }
 }
 
@@ -408,8 +433,12 @@ cudaError_t ns_gemm_prepare() {
                               kGemmSmemBytes);
 }
 
-cudaError_t launch_ns_gemm(const NsGemmParams& p, int grid, cudaStream_t s) {
-  ns_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, s>>>(p);
+cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s) {
+  const int tiles = p.tile_begin[p.nbanks];
+  int pairs = num_sms / 2;
+  if (tiles < pairs) pairs = tiles;
+  if (pairs < 1) pairs = 1;
+  ns_gemm_kernel<<<2 * pairs, kGemmThreads, kGemmSmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 

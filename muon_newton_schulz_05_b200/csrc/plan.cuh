@@ -18,12 +18,13 @@
 namespace muon {
 
 constexpr int kPad = 256;          // padding granule of R and C
-constexpr int kBM = 128;           // GEMM tile rows (UMMA M)
-constexpr int kBN = 256;           // GEMM tile cols (UMMA N)
+constexpr int kTile = 256;         // GEMM tile (rows and cols) computed by one CTA pair
+constexpr int kBM = 128;           // tile rows held by one CTA of the pair
+constexpr int kBN = 256;           // tile cols (UMMA N); each CTA loads kBN/2 of B
 constexpr int kBK = 64;            // K per pipeline stage (one 128-byte swizzle row)
-constexpr int kStages = 4;         // TMA -> MMA pipeline depth
+constexpr int kStages = 6;         // TMA -> MMA pipeline depth
 constexpr int kATileBytes = kBM * kBK * 2;
-constexpr int kBTileBytes = kBN * kBK * 2;
+constexpr int kBTileBytes = (kBN / 2) * kBK * 2;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 + 256;
 constexpr int kEpiWarps = 8;      // two per TMEM lane quadrant
@@ -39,8 +40,8 @@ enum MapSlot : int { kHiK0 = 0, kHiK1 = 1, kHiMN0 = 2, kHiMN1 = 3, kAK = 4, kBK_
 struct BankPlan {
   int count, R, C, Rp, Cp, rp, tall;
   int chunks;                   // momentum-pass blocks per matrix
-  int tiles_sym;                // upper tiles of an rp x rp symmetric product
-  int tiles_apply;              // (Rp/128) * (Cp/256)
+  int tiles_sym;                // upper 256x256 tiles of an rp x rp symmetric product
+  int tiles_apply;              // (Rp/256) * (Cp/256)
   __nv_bfloat16* hi[2];         // iterate, high bf16 part (ping-pong)
   __nv_bfloat16* lo;            // iterate, low bf16 part (in place)
   __nv_bfloat16* A;             // Gram matrix, count x rp x rp
@@ -112,7 +113,7 @@ struct UpdParams {
 // Launchers (defined in the .cu files).
 cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total_mats,
                                  cudaStream_t s);
-cudaError_t launch_ns_gemm(const NsGemmParams& p, int grid, cudaStream_t s);
+cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_update(const UpdParams& p, long long total_elems, int num_sms,
                           cudaStream_t s);
 cudaError_t launch_ema(float* ema, const void* param, int param_dtype, long long n, float beta,
