@@ -169,27 +169,43 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
   return off;
 }
 
-muon_status encode_map(CUtensorMap* m, void* ptr, int64_t inner, int64_t outer, int box_outer) {
+muon_status encode_map(CUtensorMap* m, void* ptr, int64_t inner, int64_t outer, int box_inner,
+                       int box_outer, CUtensorMapSwizzle swz) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MUON_OK : MUON_ERR_CUDA;
 }
 
 muon_status encode_bank_maps(const BankPlan& p, CUtensorMap* maps) {
   const int64_t rows = static_cast<int64_t>(p.count) * p.Rp;
   const int64_t srows = static_cast<int64_t>(p.count) * p.rp;
-  muon_status st;
-  for (int k = 0; k < 2; ++k) {
-    if ((st = encode_map(&maps[kHiK0 + k], p.hi[k], p.Cp, rows, 128)) != MUON_OK) return st;
-    if ((st = encode_map(&maps[kHiMN0 + k], p.hi[k], p.Cp, rows, 64)) != MUON_OK) return st;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B, none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  struct Spec {
+    int slot;
+    void* ptr;
+    int64_t inner, outer;
+    int bi, bo;
+    CUtensorMapSwizzle swz;
+  } specs[] = {
+      {kHiK0, p.hi[0], p.Cp, rows, 64, 128, sw},    {kHiK1, p.hi[1], p.Cp, rows, 64, 128, sw},
+      {kHiMN0, p.hi[0], p.Cp, rows, 64, 64, sw},    {kHiMN1, p.hi[1], p.Cp, rows, 64, 64, sw},
+      {kAK, p.A, p.rp, srows, 64, 128, sw},         {kBK_, p.B, p.rp, srows, 64, 128, sw},
+      {kHiE0, p.hi[0], p.Cp, rows, kEpiCols, kEpiRows, sw},
+      {kHiE1, p.hi[1], p.Cp, rows, kEpiCols, kEpiRows, sw},
+      {kLoE, p.lo, p.Cp, rows, kEpiCols, kEpiRows, sw},
+      {kAE, p.A, p.rp, srows, kEpiCols, kEpiRows, sw}, {kAT, p.A, p.rp, srows, kEpiRows, kEpiCols, none},
+      {kBE, p.B, p.rp, srows, kEpiCols, kEpiRows, sw}, {kBT, p.B, p.rp, srows, kEpiRows, kEpiCols, none},
+  };
+  for (const Spec& sp : specs) {
+    muon_status st = encode_map(&maps[sp.slot], sp.ptr, sp.inner, sp.outer, sp.bi, sp.bo, sp.swz);
+    if (st != MUON_OK) return st;
   }
-  if ((st = encode_map(&maps[kAK], p.A, p.rp, srows, 128)) != MUON_OK) return st;
-  return encode_map(&maps[kBK_], p.B, p.rp, srows, 128);
+  return MUON_OK;
 }
 
 // ------------------------------------------------------------ the step

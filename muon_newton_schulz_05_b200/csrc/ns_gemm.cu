@@ -120,88 +120,53 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_majo
 }
 
 // ---------------------------------------------------------------- epilogues
-// Each epilogue thread owns one accumulator row and handles 64 columns at a
-// time: its global inputs (the previous iterate for Apply, A for Poly) are
-// loaded first, then two 32-column TMEM loads share one wait.
-struct EpiIn {
-  uint4 x[8];  // Apply: hi of 64 columns; Poly: A of 64 columns
-  uint4 y[8];  // Apply: lo of 64 columns
+// Each epilogue warp owns 32 accumulator rows and 128 of the 256 columns and
+// works on 32 x 64 chunks. Global traffic goes through TMA only: the chunk's
+// inputs (Apply: hi and lo of the iterate; Poly: A) are bulk-loaded into two
+// 4 KB per-warp buffers, the results are written back into the buffers and
+// bulk-stored. Row-wise buffers use the 128-byte swizzle of the TMA box
+// (16-byte group g of row r at r*128 + ((g ^ (r & 7)) * 16), base 1 KB
+// aligned), so a lane reading or writing its own row touches 8 distinct
+// bank groups per quarter warp. The transposed mirror chunk of an
+// off-diagonal Gram/Poly tile is a plain [64][32] buffer written one column
+// (64 contiguous bytes across the warp) at a time.
+__device__ __forceinline__ uint32_t swz_off(int r, int g) {
+  return static_cast<uint32_t>(r * 128 + ((g ^ (r & 7)) << 4));
+}
+
+struct EpiCtx {
+  uint8_t* bufA;   // swizzled [32][64] bf16: hi (Apply), A in / out (Poly), out (Gram)
+  uint8_t* bufB;   // swizzled [32][64] lo (Apply) or plain [64][32] mirror (Gram / Poly)
+  uint64_t* bar;   // this warp's load barrier
+  uint32_t phase;  // its parity
 };
 
-__device__ __forceinline__ void epi_prefetch(const NsGemmParams& p, const BankPlan& bp, int mat,
-                                             int row, int col0, EpiIn& in) {
-  if (p.phase == kApply) {
-    const size_t off = static_cast<size_t>(mat) * bp.Rp * bp.Cp + static_cast<size_t>(row) * bp.Cp + col0;
-    const uint4* hin = reinterpret_cast<const uint4*>(bp.hi[p.cur] + off);
-    const uint4* lio = reinterpret_cast<const uint4*>(bp.lo + off);
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      in.x[g] = hin[g];
-      in.y[g] = lio[g];
+// Bulk-load the chunk's inputs (lane 0 issues, every lane waits). False if the
+// wait gave up.
+__device__ __forceinline__ bool epi_load(const NsGemmParams& p, EpiCtx& e, const Tile& T,
+                                         const BankPlan& bp, int r0, int c0, int lane,
+                                         volatile int* abort_flag) {
+  if (p.phase == kGram) return true;
+  if (lane == 0) {
+    if (p.phase == kApply) {
+      const int y = T.mat * bp.Rp + r0;
+      mbar_arrive_expect_tx(e.bar, 2 * kEpiRows * kEpiCols * 2);
+      tma_load_2d(e.bufA, &p.maps[T.bank][kHiE0 + p.cur], e.bar, c0, y);
+      tma_load_2d(e.bufB, &p.maps[T.bank][kLoE], e.bar, c0, y);
+    } else {
+      mbar_arrive_expect_tx(e.bar, kEpiRows * kEpiCols * 2);
+      tma_load_2d(e.bufA, &p.maps[T.bank][kAE], e.bar, c0, T.mat * bp.rp + r0);
     }
-  } else if (p.phase == kPoly && col0 + 63 >= row) {
-    const size_t rp = static_cast<size_t>(bp.rp);
-    const uint4* ain = reinterpret_cast<const uint4*>(bp.A + static_cast<size_t>(mat) * rp * rp + row * rp + col0);
-#pragma unroll
-    for (int g = 0; g < 8; ++g) in.x[g] = ain[g];
   }
+  const bool ok = mbar_wait(e.bar, e.phase, abort_flag, p.status, p.wait_limit_ns);
+  e.phase ^= 1u;
+  return __all_sync(0xffffffffu, ok);
 }
 
-// Gram / Poly: columns col0 .. col0+31 of row `row` in v[]; a4 = A there (Poly).
-// Stores the upper part (col >= row) in place and mirrors the strict upper part.
-__device__ __forceinline__ void epilogue_sym(const NsGemmParams& p, const BankPlan& bp, int mat,
-                                             int row, int col0, float (&v)[32], const uint4* a4) {
-  if (col0 + 31 < row) return;  // entirely below the diagonal: the mirror covers it
-  const size_t rp = static_cast<size_t>(bp.rp);
-  const size_t mbase = static_cast<size_t>(mat) * rp * rp;
-  __nv_bfloat16* out = (p.phase == kGram ? bp.A : bp.B) + mbase;
-  if (p.phase == kGram) {
-    if (p.iter == 0) {  // the operand holds U; fold 1 / ||U||^2 in here
-      const float s = bp.scale[mat];
-      const float s2 = s * s;
-#pragma unroll
-      for (int t = 0; t < 32; ++t) v[t] *= s2;
-    }
-  } else {
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const uint32_t ww[4] = {a4[g].x, a4[g].y, a4[g].z, a4[g].w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        v[8 * g + 2 * h] = fmaf(p.c, v[8 * g + 2 * h], p.b * bf16_lo_f(ww[h]));
-        v[8 * g + 2 * h + 1] = fmaf(p.c, v[8 * g + 2 * h + 1], p.b * bf16_hi_f(ww[h]));
-      }
-    }
-  }
-  uint32_t pk[16];
-#pragma unroll
-  for (int h = 0; h < 16; ++h) pk[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
-  __nv_bfloat16* orow = out + row * rp + col0;
-  if (col0 >= row) {
-    uint4* o4 = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-    for (int g = 0; g < 4; ++g) o4[g] = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
-  } else {
-    const unsigned short* ps = reinterpret_cast<const unsigned short*>(pk);
-#pragma unroll
-    for (int t = 0; t < 32; ++t)
-      if (col0 + t >= row) reinterpret_cast<unsigned short*>(orow)[t] = ps[t];
-  }
-  const unsigned short* ps = reinterpret_cast<const unsigned short*>(pk);
-  unsigned short* ocol = reinterpret_cast<unsigned short*>(out + static_cast<size_t>(col0) * rp + row);
-#pragma unroll
-  for (int t = 0; t < 32; ++t)
-    if (col0 + t > row) ocol[static_cast<size_t>(t) * rp] = ps[t];
-}
-
-// Apply: x' = alpha x + beta D with x = hi + lo (h4, l4: 32 columns);
-// writes hi' (other buffer) and lo.
-__device__ __forceinline__ void epilogue_apply(const NsGemmParams& p, const BankPlan& bp, int mat,
-                                               int row, int col0, const float (&v)[32],
-                                               const uint4* h4, const uint4* l4) {
-  const size_t off = static_cast<size_t>(mat) * bp.Rp * bp.Cp + static_cast<size_t>(row) * bp.Cp + col0;
-  uint4* hout = reinterpret_cast<uint4*>(bp.hi[p.cur ^ 1] + off);
-  uint4* lio = reinterpret_cast<uint4*>(bp.lo + off);
+// Apply: x' = alpha x + beta D with x = hi + lo, for this lane's row of the chunk.
+__device__ __forceinline__ void epi_apply(const NsGemmParams& p, const BankPlan& bp, int mat,
+                                          const EpiCtx& e, int lane, const uint32_t (&r0)[32],
+                                          const uint32_t (&r1)[32]) {
   float alpha = p.a, beta = 1.0f;
   if (p.iter == 0) {  // the iterate holds U; X0 = s U
     const float s = bp.scale[mat];
@@ -209,34 +174,91 @@ __device__ __forceinline__ void epilogue_apply(const NsGemmParams& p, const Bank
     beta = s;
   }
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const uint32_t hw[4] = {h4[g].x, h4[g].y, h4[g].z, h4[g].w};
-    const uint32_t lw[4] = {l4[g].x, l4[g].y, l4[g].z, l4[g].w};
+  for (int g = 0; g < 8; ++g) {
+    const uint32_t off = swz_off(lane, g);
+    const uint4 h4 = *reinterpret_cast<const uint4*>(e.bufA + off);
+    const uint4 l4 = *reinterpret_cast<const uint4*>(e.bufB + off);
+    const uint32_t hw[4] = {h4.x, h4.y, h4.z, h4.w};
+    const uint32_t lw[4] = {l4.x, l4.y, l4.z, l4.w};
     uint32_t ho[4], lo[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      const float x0 = bf16_lo_f(hw[h]) + bf16_lo_f(lw[h]);
-      const float x1 = bf16_hi_f(hw[h]) + bf16_hi_f(lw[h]);
-      const float y0 = fmaf(alpha, x0, beta * v[8 * g + 2 * h]);
-      const float y1 = fmaf(alpha, x1, beta * v[8 * g + 2 * h + 1]);
+      const int c = 8 * g + 2 * h;
+      const float d0 = __uint_as_float(c < 32 ? r0[c & 31] : r1[c & 31]);
+      const float d1 = __uint_as_float(c + 1 < 32 ? r0[(c + 1) & 31] : r1[(c + 1) & 31]);
+      const float y0 = fmaf(alpha, bf16_lo_f(hw[h]) + bf16_lo_f(lw[h]), beta * d0);
+      const float y1 = fmaf(alpha, bf16_hi_f(hw[h]) + bf16_hi_f(lw[h]), beta * d1);
       ho[h] = pack_bf16x2(y0, y1);
       lo[h] = pack_bf16x2(y0 - bf16_lo_f(ho[h]), y1 - bf16_hi_f(ho[h]));
     }
-    hout[g] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
-    lio[g] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4*>(e.bufA + off) = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+    *reinterpret_cast<uint4*>(e.bufB + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
-__device__ __forceinline__ void epilogue_chunk(const NsGemmParams& p, const BankPlan& bp, int mat,
-                                               int row, int col0, const uint32_t (&r)[32],
-                                               const EpiIn& in, int part) {
-  float v[32];
+// Gram (A = D, times s^2 at step 0) or Poly (B = b A + c D) for this lane's
+// row; the transposed copy goes to the mirror buffer when `mirror`.
+__device__ __forceinline__ void epi_sym(const NsGemmParams& p, const BankPlan& bp, int mat,
+                                        const EpiCtx& e, int lane, bool mirror,
+                                        const uint32_t (&r0)[32], const uint32_t (&r1)[32]) {
+  float scl = 1.0f;
+  if (p.phase == kGram && p.iter == 0) {  // the operand holds U; fold 1 / ||U||^2 in here
+    const float s = bp.scale[mat];
+    scl = s * s;
+  }
+  unsigned short* mir = reinterpret_cast<unsigned short*>(e.bufB);
 #pragma unroll
-  for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
-  if (p.phase == kApply)
-    epilogue_apply(p, bp, mat, row, col0, v, in.x + 4 * part, in.y + 4 * part);
-  else
-    epilogue_sym(p, bp, mat, row, col0, v, in.x + 4 * part);
+  for (int g = 0; g < 8; ++g) {
+    const uint32_t off = swz_off(lane, g);
+    float v[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int c = 8 * g + t;
+      v[t] = __uint_as_float(c < 32 ? r0[c & 31] : r1[c & 31]);
+    }
+    if (p.phase == kPoly) {
+      const uint4 a4 = *reinterpret_cast<const uint4*>(e.bufA + off);
+      const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        v[2 * h] = fmaf(p.c, v[2 * h], p.b * bf16_lo_f(aw[h]));
+        v[2 * h + 1] = fmaf(p.c, v[2 * h + 1], p.b * bf16_hi_f(aw[h]));
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[t] *= scl;
+    }
+    uint32_t pk[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) pk[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
+    *reinterpret_cast<uint4*>(e.bufA + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    if (mirror) {
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        mir[(8 * g + 2 * h) * kEpiRows + lane] = static_cast<unsigned short>(pk[h] & 0xFFFFu);
+        mir[(8 * g + 2 * h + 1) * kEpiRows + lane] = static_cast<unsigned short>(pk[h] >> 16);
+      }
+    }
+  }
+}
+
+// Bulk-store the chunk (lane 0, after every lane's writes are visible to TMA).
+__device__ __forceinline__ void epi_store(const NsGemmParams& p, const EpiCtx& e, const Tile& T,
+                                          const BankPlan& bp, int r0, int c0, int lane, bool mirror) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    if (p.phase == kApply) {
+      const int y = T.mat * bp.Rp + r0;
+      tma_store_2d(&p.maps[T.bank][kHiE0 + (p.cur ^ 1)], e.bufA, c0, y);
+      tma_store_2d(&p.maps[T.bank][kLoE], e.bufB, c0, y);
+    } else {
+      const int base = T.mat * bp.rp;
+      tma_store_2d(&p.maps[T.bank][p.phase == kGram ? kAE : kBE], e.bufA, c0, base + r0);
+      if (mirror) tma_store_2d(&p.maps[T.bank][p.phase == kGram ? kAT : kBT], e.bufB, r0, base + c0);
+    }
+    bulk_commit();
+  }
 }
 
 // Waits that ignore the abort flag, used only to drain in-flight work.
@@ -253,12 +275,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* epibuf = smem + kStages * kStageBytes;  // kEpiWarps x kEpiBufBytes, 1 KB aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(epibuf + kEpiWarps * kEpiBufBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* epibar = done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + kEpiWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -279,6 +303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 2 * kEpiWarps);  // the leader's: both CTAs' epilogue warps
     }
     mbar_init(done, 1);
+    for (int w = 0; w < kEpiWarps; ++w) mbar_init(&epibar[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -384,15 +409,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // 2..5 take accumulator columns 0..127 and warps 6..9 columns 128..255.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
+    const int ew = warp - 2;
+    EpiCtx e{epibuf + ew * kEpiBufBytes, epibuf + ew * kEpiBufBytes + kEpiBufBytes / 2, &epibar[ew], 0u};
     const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = pair; tile < ntiles; tile += npairs) {
+    bool ok = true;
+    for (int tile = pair; ok && tile < ntiles; tile += npairs) {
       const Tile T = decode_tile(p, tile);
       const BankPlan& bp = p.bank[T.bank];
-      const int row = T.m0 + kBM * static_cast<int>(rank) + 32 * q + lane;
-      EpiIn in;
-      epi_prefetch(p, bp, T.mat, row, T.n0 + half * 128, in);
+      const int r0 = T.m0 + kBM * static_cast<int>(rank) + 32 * q;  // first row of this warp
+      const bool mirror = p.phase != kApply && T.n0 != T.m0;
       // the tcgen05.ld below is warp-collective: leave only if the whole warp does
       const bool got = mbar_wait_cluster(&tfull[acc], acc_phase, abort_flag, p.status, limit);
       if (!__all_sync(0xffffffffu, got)) break;
@@ -401,14 +428,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                           static_cast<uint32_t>(acc * kBN + half * 128);
 #pragma unroll 1
       for (int jj = 0; jj < 2; ++jj) {
-        const int col0 = T.n0 + half * 128 + jj * 64;
-        if (jj > 0) epi_prefetch(p, bp, T.mat, row, col0, in);
-        uint32_t r0[32], r1[32];
-        tmem_ld32(tb + jj * 64, r0);
-        tmem_ld32(tb + jj * 64 + 32, r1);
+        const int c0 = T.n0 + half * 128 + jj * kEpiCols;
+        if (lane == 0) bulk_wait_read();  // the buffers' previous stores have read them
+        __syncwarp();
+        if (!epi_load(p, e, T, bp, r0, c0, lane, abort_flag)) { ok = false; break; }
+        uint32_t ra[32], rb[32];
+        tmem_ld32(tb + jj * kEpiCols, ra);
+        tmem_ld32(tb + jj * kEpiCols + 32, rb);
         tmem_ld_wait();
-        epilogue_chunk(p, bp, T.mat, row, col0, r0, in, 0);
-        epilogue_chunk(p, bp, T.mat, row, col0 + 32, r1, in, 1);
+        if (p.phase == kApply)
+          epi_apply(p, bp, T.mat, e, lane, ra, rb);
+        else
+          epi_sym(p, bp, T.mat, e, lane, mirror, ra, rb);
+        epi_store(p, e, T, bp, r0, c0, lane, mirror);
       }
       tc_fence_before();
       __syncwarp();
@@ -416,6 +448,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();  // every bulk store of this warp has completed
+    __syncwarp();
   }
 
   tc_fence_before();
