@@ -155,6 +155,7 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
     const size_t o_A = take(sq_bytes), o_B = take(sq_bytes);
     const size_t o_part = take(static_cast<size_t>(p.count) * p.chunks * 4);
     const size_t o_scale = take(static_cast<size_t>(p.count) * 4);
+    const size_t o_cnt = take(static_cast<size_t>(p.count) * 3 * 4);
     if (base) {
       p.hi[0] = reinterpret_cast<__nv_bfloat16*>(base + o_hi0);
       p.hi[1] = reinterpret_cast<__nv_bfloat16*>(base + o_hi1);
@@ -163,6 +164,7 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
       p.B = reinterpret_cast<__nv_bfloat16*>(base + o_B);
       p.partial = reinterpret_cast<float*>(base + o_part);
       p.scale = reinterpret_cast<float*>(base + o_scale);
+      p.counters = reinterpret_cast<int*>(base + o_cnt);
       plans[b] = p;
     }
   }
@@ -276,23 +278,18 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
     std::swap(ev_after, g_ev_after);
   }
   if (ev_before && cudaEventRecord(ev_before, stream) != cudaSuccess) return MUON_ERR_CUDA;
-  for (int it = 0; it < hp->ns_steps; ++it) {
-    gp.iter = it;
-    gp.cur = it & 1;
-    gp.a = hp->coeffs[3 * it];
-    gp.b = hp->coeffs[3 * it + 1];
-    gp.c = hp->coeffs[3 * it + 2];
-    for (int ph = kGram; ph <= kApply; ++ph) {
-      gp.phase = ph;
-      int tiles = 0;
-      for (int b = 0; b < nbanks; ++b) {
-        gp.tile_begin[b] = tiles;
-        tiles += plans[b].count * (ph == kApply ? plans[b].tiles_apply : plans[b].tiles_sym);
-      }
-      gp.tile_begin[nbanks] = tiles;
-      if (launch_ns_gemm(gp, sms, stream) != cudaSuccess) return MUON_ERR_CUDA;
-    }
+  gp.ns_steps = hp->ns_steps;
+  for (int i = 0; i < 3 * hp->ns_steps; ++i) gp.coef[i] = hp->coeffs[i];
+  int sym = 0, app = 0;
+  for (int b = 0; b < nbanks; ++b) {
+    gp.sym_begin[b] = sym;
+    gp.apply_begin[b] = app;
+    sym += plans[b].count * plans[b].tiles_sym;
+    app += plans[b].count * plans[b].tiles_apply;
   }
+  gp.sym_begin[nbanks] = sym;
+  gp.apply_begin[nbanks] = app;
+  if (launch_ns_gemm(gp, sms, stream) != cudaSuccess) return MUON_ERR_CUDA;
   if (ev_after && cudaEventRecord(ev_after, stream) != cudaSuccess) return MUON_ERR_CUDA;
 
   // ---- scale, decay, parameter write (+ EMA), or O out

@@ -3,7 +3,8 @@
 //                   ANVIL momenta), writes U as the bf16 hi/lo iterate in the
 //                   padded working layout and per-block partial sums of U^2
 //   norm_finalize : 1 / (||U||_F + eps) per matrix from the partials, in a
-//                   fixed order (deterministic)
+//                   fixed order (deterministic); resets the matrix's
+//                   Newton-Schulz completion counters
 //   update        : theta <- theta (1 - lr wd [mask]) - lr s O, optional EMA
 //   ema / blend   : standalone EMA and readout blend
 // ("Muonとは": momentum as a moving average of the gradient; "ANVIL II와 가중치
@@ -180,6 +181,8 @@ __global__ void __launch_bounds__(128) norm_finalize_kernel(const __grid_constan
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) bp.scale[mat] = static_cast<float>(1.0 / (sqrt(s) + static_cast<double>(p.eps)));
+  // the Newton-Schulz chain's per-matrix completion counters start at zero
+  if (lane < 3) bp.counters[3 * mat + lane] = 0;
 }
 
 cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total_mats,

@@ -1,6 +1,7 @@
 // Newton-Schulz GEMM chain on sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// One persistent launch per (step, phase). The three phases of a step are
+// One persistent launch runs the whole chain: every step and phase of every
+// matrix of every bank (see NsGemmParams). The three phases of a step are
 //   Gram : A = X X^T            (tall: A = Y^T Y)      upper tiles only, mirrored
 //   Poly : B = b A + c A A      (A symmetric)          upper tiles only, mirrored
 //   Apply: X <- a X + B X       (tall: Y <- a Y + Y B) full tiles
@@ -32,8 +33,13 @@ namespace muon {
 
 struct Tile {
   int bank, mat, m0, n0, nkb;
+  int phase, iter, cur;       // Phase, Newton-Schulz step, hi buffer holding X_iter
+  float a, b, c;              // this step's coefficients
   int a_map, a_mn, a_base;
   int b_map, b_mn, b_base;
+  int* done_cnt;              // counter this tile's epilogue advances
+  const int* dep_cnt;         // counter of the phase this tile reads
+  int dep_target;             // value dep_cnt must reach first (0: nothing to wait for)
 };
 
 // Upper 256 x 256 tiles (diagonal included) of a symmetric product with nb
@@ -50,12 +56,33 @@ __device__ __forceinline__ void sym_tile(int t, int nb, int& i, int& j) {
 
 __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   Tile T;
+  const int S = p.sym_begin[p.nbanks];
+  const int per_iter = 2 * S + p.apply_begin[p.nbanks];
+  T.iter = tile / per_iter;
+  int r = tile - T.iter * per_iter;
+  const int* begin;
+  if (r < S) {
+    T.phase = kGram;
+    begin = p.sym_begin;
+  } else if (r < 2 * S) {
+    T.phase = kPoly;
+    r -= S;
+    begin = p.sym_begin;
+  } else {
+    T.phase = kApply;
+    r -= 2 * S;
+    begin = p.apply_begin;
+  }
   int b = 0;
-  while (b + 1 < p.nbanks && tile >= p.tile_begin[b + 1]) ++b;
+  while (b + 1 < p.nbanks && r >= begin[b + 1]) ++b;
   const BankPlan& bp = p.bank[b];
-  const int local = tile - p.tile_begin[b];
+  const int local = r - begin[b];
   T.bank = b;
-  if (p.phase == kApply) {
+  T.cur = T.iter & 1;
+  T.a = p.coef[3 * T.iter];
+  T.b = p.coef[3 * T.iter + 1];
+  T.c = p.coef[3 * T.iter + 2];
+  if (T.phase == kApply) {
     T.mat = local / bp.tiles_apply;
     const int t = local - T.mat * bp.tiles_apply;
     const int nbn = bp.Cp / kTile;
@@ -69,10 +96,21 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
     T.m0 = i * kTile;
     T.n0 = j * kTile;
   }
-  const int cur = p.cur;
+  // Gram(k) reads X_k (all of Apply(k-1)); Poly(k) reads A (all of Gram(k));
+  // Apply(k) reads B (all of Poly(k)). Earlier phases are implied by these.
+  int* cnt = bp.counters + 3 * T.mat;
+  T.done_cnt = cnt + T.phase;
+  if (T.phase == kGram) {
+    T.dep_cnt = cnt + kApply;
+    T.dep_target = kTileParts * bp.tiles_apply * T.iter;
+  } else {
+    T.dep_cnt = cnt + (T.phase - 1);
+    T.dep_target = kTileParts * bp.tiles_sym * (T.iter + 1);
+  }
+  const int cur = T.cur;
   const int xbase = T.mat * bp.Rp;   // first row of this matrix in the iterate maps
   const int sbase = T.mat * bp.rp;   // first row of this matrix in the A / B maps
-  if (p.phase == kGram) {
+  if (T.phase == kGram) {
     if (!bp.tall) {  // D[m][n] = sum_k X[m][k] X[n][k]
       T.a_map = kHiK0 + cur; T.a_mn = 0; T.a_base = xbase;
       T.b_map = kHiK0 + cur; T.b_mn = 0; T.b_base = xbase;
@@ -82,7 +120,7 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
       T.b_map = kHiMN0 + cur; T.b_mn = 1; T.b_base = xbase;
       T.nkb = bp.Rp / kBK;
     }
-  } else if (p.phase == kPoly) {  // D[m][n] = sum_k A[m][k] A[n][k]
+  } else if (T.phase == kPoly) {  // D[m][n] = sum_k A[m][k] A[n][k]
     T.a_map = kAK; T.a_mn = 0; T.a_base = sbase;
     T.b_map = kAK; T.b_mn = 0; T.b_base = sbase;
     T.nkb = bp.rp / kBK;
@@ -98,6 +136,29 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
     }
   }
   return T;
+}
+
+// Bounded wait until *cnt >= target (acquire, GPU scope), then order the
+// async-proxy (TMA) reads that follow after it. False if it gave up.
+__device__ __forceinline__ bool wait_dependency(const int* cnt, int target, volatile int* abort,
+                                                int* status, uint64_t limit_ns) {
+  if (target > 0 && ld_acquire_gpu(cnt) < target) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+      __nanosleep(64);
+      if (ld_acquire_gpu(cnt) >= target) break;
+      if ((i & 15u) == 0) {
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+          *abort = 1;
+          atomicExch(status, 8 /* MUON_ERR_TIMEOUT */);
+          return false;
+        }
+      }
+    }
+  }
+  fence_proxy_async_global();
+  return true;
 }
 
 // This CTA's 128 (MN) x 64 (K) slice of an operand tile into dst; completion
@@ -146,12 +207,12 @@ struct EpiCtx {
 __device__ __forceinline__ bool epi_load(const NsGemmParams& p, EpiCtx& e, const Tile& T,
                                          const BankPlan& bp, int r0, int c0, int lane,
                                          volatile int* abort_flag) {
-  if (p.phase == kGram) return true;
+  if (T.phase == kGram) return true;
   if (lane == 0) {
-    if (p.phase == kApply) {
+    if (T.phase == kApply) {
       const int y = T.mat * bp.Rp + r0;
       mbar_arrive_expect_tx(e.bar, 2 * kEpiRows * kEpiCols * 2);
-      tma_load_2d(e.bufA, &p.maps[T.bank][kHiE0 + p.cur], e.bar, c0, y);
+      tma_load_2d(e.bufA, &p.maps[T.bank][kHiE0 + T.cur], e.bar, c0, y);
       tma_load_2d(e.bufB, &p.maps[T.bank][kLoE], e.bar, c0, y);
     } else {
       mbar_arrive_expect_tx(e.bar, kEpiRows * kEpiCols * 2);
@@ -164,12 +225,12 @@ __device__ __forceinline__ bool epi_load(const NsGemmParams& p, EpiCtx& e, const
 }
 
 // Apply: x' = alpha x + beta D with x = hi + lo, for this lane's row of the chunk.
-__device__ __forceinline__ void epi_apply(const NsGemmParams& p, const BankPlan& bp, int mat,
-                                          const EpiCtx& e, int lane, const uint32_t (&r0)[32],
+__device__ __forceinline__ void epi_apply(const Tile& T, const BankPlan& bp, const EpiCtx& e,
+                                          int lane, const uint32_t (&r0)[32],
                                           const uint32_t (&r1)[32]) {
-  float alpha = p.a, beta = 1.0f;
-  if (p.iter == 0) {  // the iterate holds U; X0 = s U
-    const float s = bp.scale[mat];
+  float alpha = T.a, beta = 1.0f;
+  if (T.iter == 0) {  // the iterate holds U; X0 = s U
+    const float s = bp.scale[T.mat];
     alpha *= s;
     beta = s;
   }
@@ -198,12 +259,12 @@ __device__ __forceinline__ void epi_apply(const NsGemmParams& p, const BankPlan&
 
 // Gram (A = D, times s^2 at step 0) or Poly (B = b A + c D) for this lane's
 // row; the transposed copy goes to the mirror buffer when `mirror`.
-__device__ __forceinline__ void epi_sym(const NsGemmParams& p, const BankPlan& bp, int mat,
-                                        const EpiCtx& e, int lane, bool mirror,
-                                        const uint32_t (&r0)[32], const uint32_t (&r1)[32]) {
+__device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, const EpiCtx& e,
+                                        int lane, bool mirror, const uint32_t (&r0)[32],
+                                        const uint32_t (&r1)[32]) {
   float scl = 1.0f;
-  if (p.phase == kGram && p.iter == 0) {  // the operand holds U; fold 1 / ||U||^2 in here
-    const float s = bp.scale[mat];
+  if (T.phase == kGram && T.iter == 0) {  // the operand holds U; fold 1 / ||U||^2 in here
+    const float s = bp.scale[T.mat];
     scl = s * s;
   }
   unsigned short* mir = reinterpret_cast<unsigned short*>(e.bufB);
@@ -216,13 +277,13 @@ __device__ __forceinline__ void epi_sym(const NsGemmParams& p, const BankPlan& b
       const int c = 8 * g + t;
       v[t] = __uint_as_float(c < 32 ? r0[c & 31] : r1[c & 31]);
     }
-    if (p.phase == kPoly) {
+    if (T.phase == kPoly) {
       const uint4 a4 = *reinterpret_cast<const uint4*>(e.bufA + off);
       const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        v[2 * h] = fmaf(p.c, v[2 * h], p.b * bf16_lo_f(aw[h]));
-        v[2 * h + 1] = fmaf(p.c, v[2 * h + 1], p.b * bf16_hi_f(aw[h]));
+        v[2 * h] = fmaf(T.c, v[2 * h], T.b * bf16_lo_f(aw[h]));
+        v[2 * h + 1] = fmaf(T.c, v[2 * h + 1], T.b * bf16_hi_f(aw[h]));
       }
     } else {
 #pragma unroll
@@ -248,14 +309,14 @@ __device__ __forceinline__ void epi_store(const NsGemmParams& p, const EpiCtx& e
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    if (p.phase == kApply) {
+    if (T.phase == kApply) {
       const int y = T.mat * bp.Rp + r0;
-      tma_store_2d(&p.maps[T.bank][kHiE0 + (p.cur ^ 1)], e.bufA, c0, y);
+      tma_store_2d(&p.maps[T.bank][kHiE0 + (T.cur ^ 1)], e.bufA, c0, y);
       tma_store_2d(&p.maps[T.bank][kLoE], e.bufB, c0, y);
     } else {
       const int base = T.mat * bp.rp;
-      tma_store_2d(&p.maps[T.bank][p.phase == kGram ? kAE : kBE], e.bufA, c0, base + r0);
-      if (mirror) tma_store_2d(&p.maps[T.bank][p.phase == kGram ? kAT : kBT], e.bufB, r0, base + c0);
+      tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAE : kBE], e.bufA, c0, base + r0);
+      if (mirror) tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAT : kBT], e.bufB, r0, base + c0);
     }
     bulk_commit();
   }
@@ -291,7 +352,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t rank = cluster_ctarank();  // 0: pair leader, issues the MMAs
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
-  const int ntiles = p.tile_begin[p.nbanks];
+  const int ntiles = p.ns_steps * (2 * p.sym_begin[p.nbanks] + p.apply_begin[p.nbanks]);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -335,6 +396,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const Tile T = decode_tile(p, tile);
         const CUtensorMap* amap = &p.maps[T.bank][T.a_map];
         const CUtensorMap* bmap = &p.maps[T.bank][T.b_map];
+        // the operands of this tile are final once the phase it reads is done
+        if (!wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) {
+          ok = false;
+          break;
+        }
         for (int kb = 0; kb < T.nkb; ++kb) {
           if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, abort_flag, p.status, limit)) {
             ok = false;
@@ -419,7 +485,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const Tile T = decode_tile(p, tile);
       const BankPlan& bp = p.bank[T.bank];
       const int r0 = T.m0 + kBM * static_cast<int>(rank) + 32 * q;  // first row of this warp
-      const bool mirror = p.phase != kApply && T.n0 != T.m0;
+      const bool mirror = T.phase != kApply && T.n0 != T.m0;
+      // the epilogue's own TMA loads read the same finished phase
+      if (lane == 0 && T.phase != kGram &&
+          !wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit))
+        ok = false;
+      if (!__all_sync(0xffffffffu, ok)) break;
       // the tcgen05.ld below is warp-collective: leave only if the whole warp does
       const bool got = mbar_wait_cluster(&tfull[acc], acc_phase, abort_flag, p.status, limit);
       if (!__all_sync(0xffffffffu, got)) break;
@@ -436,15 +507,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(tb + jj * kEpiCols, ra);
         tmem_ld32(tb + jj * kEpiCols + 32, rb);
         tmem_ld_wait();
-        if (p.phase == kApply)
-          epi_apply(p, bp, T.mat, e, lane, ra, rb);
+        if (T.phase == kApply)
+          epi_apply(T, bp, e, lane, ra, rb);
         else
-          epi_sym(p, bp, T.mat, e, lane, mirror, ra, rb);
+          epi_sym(T, bp, e, lane, mirror, ra, rb);
         epi_store(p, e, T, bp, r0, c0, lane, mirror);
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
+      if (lane == 0) {
+        mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
+        // this warp's part of the tile is in global memory: publish it
+        bulk_wait_all();
+        fence_proxy_async_global();
+        red_release_gpu_add(T.done_cnt, 1);
+      }
+      __syncwarp();
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -468,7 +547,7 @@ cudaError_t ns_gemm_prepare() {
 }
 
 cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s) {
-  const int tiles = p.tile_begin[p.nbanks];
+  const int tiles = p.ns_steps * (2 * p.sym_begin[p.nbanks] + p.apply_begin[p.nbanks]);
   int pairs = num_sms / 2;
   if (tiles < pairs) pairs = tiles;
   if (pairs < 1) pairs = 1;

@@ -57,21 +57,28 @@ struct BankPlan {
   __nv_bfloat16* B;             // b A + c A^2, count x rp x rp
   float* partial;               // count x chunks sums of squares
   float* scale;                 // count: 1 / (||U||_F + eps)
+  int* counters;                // count x 3: finished tile parts of Gram, Poly, Apply
 };
 
 // ---------------------------------------------------------------- GEMM chain
+// One persistent launch runs every Newton-Schulz step of every matrix. Tiles
+// are listed step by step, phase by phase, bank by bank, matrix by matrix;
+// CTA pairs take them round-robin. A tile waits on per-matrix counters for
+// the phase it reads; every epilogue warp of both CTAs adds 1 to its own
+// phase's counter when its stores are complete (kTileParts per tile).
+constexpr int kTileParts = 2 * kEpiWarps;
+
 struct NsGemmParams {
   CUtensorMap maps[MUON_MAX_BANKS][kMaxMaps];
   BankPlan bank[MUON_MAX_BANKS];
-  int tile_begin[MUON_MAX_BANKS + 1];
+  int sym_begin[MUON_MAX_BANKS + 1];    // prefix sums of count * tiles_sym
+  int apply_begin[MUON_MAX_BANKS + 1];  // prefix sums of count * tiles_apply
   int nbanks;
-  int phase;          // Phase
-  int iter;           // 0-based Newton-Schulz step
-  int cur;            // hi buffer holding the current iterate
-  float a, b, c;      // this step's coefficients
-  int* status;        // device status word
+  int ns_steps;
+  float coef[3 * MUON_MAX_NS_STEPS];    // (a, b, c) per step
+  int* status;                          // device status word
   unsigned long long wait_limit_ns;
-  int fault;          // test hook (muon_set_debug)
+  int fault;                            // test hook (muon_set_debug)
 };
 
 // ---------------------------------------------------------- momentum + norm
@@ -122,7 +129,7 @@ struct UpdParams {
 // Launchers (defined in the .cu files).
 cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total_mats,
                                  cudaStream_t s);
-cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s);
+cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s);  // whole chain
 cudaError_t launch_update(const UpdParams& p, long long total_elems, int num_sms,
                           cudaStream_t s);
 cudaError_t launch_ema(float* ema, const void* param, int param_dtype, long long n, float beta,
