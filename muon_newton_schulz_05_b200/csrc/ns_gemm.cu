@@ -182,52 +182,59 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_majo
 
 // ---------------------------------------------------------------- epilogues
 // Each epilogue warp owns 32 accumulator rows and 128 of the 256 columns and
-// works on 32 x 64 chunks. Global traffic goes through TMA only: the chunk's
-// inputs (Apply: hi and lo of the iterate; Poly: A) are bulk-loaded into two
-// 4 KB per-warp buffers, the results are written back into the buffers and
-// bulk-stored. Row-wise buffers use the 128-byte swizzle of the TMA box
-// (16-byte group g of row r at r*128 + ((g ^ (r & 7)) * 16), base 1 KB
-// aligned), so a lane reading or writing its own row touches 8 distinct
-// bank groups per quarter warp. The transposed mirror chunk of an
-// off-diagonal Gram/Poly tile is a plain [64][32] buffer written one column
-// (64 contiguous bytes across the warp) at a time.
-__device__ __forceinline__ uint32_t swz_off(int r, int g) {
-  return static_cast<uint32_t>(r * 128 + ((g ^ (r & 7)) << 4));
+// works through them in 32 x 32 chunks. Global traffic goes through TMA only,
+// through a ring of kEpiBufs chunk buffers per warp: while chunk j is being
+// computed, the bulk load of chunk j+1's inputs (Apply: hi and lo of the
+// iterate; Poly: A) is in flight, and the stores of earlier chunks drain.
+// Row-wise halves use the 64-byte swizzle of the TMA box (16-byte group g of
+// row r at r*64 + ((g ^ ((r >> 1) & 3)) * 16)), so a lane reading or writing
+// its own row touches 8 distinct bank groups per quarter warp. The transposed
+// mirror half of an off-diagonal Gram/Poly chunk is a plain [32][32] array
+// written one column (64 contiguous bytes across the warp) at a time.
+__device__ __forceinline__ uint32_t swz64_off(int r, int g) {
+  return static_cast<uint32_t>(r * 64 + ((g ^ ((r >> 1) & 3)) << 4));
 }
 
-struct EpiCtx {
-  uint8_t* bufA;   // swizzled [32][64] bf16: hi (Apply), A in / out (Poly), out (Gram)
-  uint8_t* bufB;   // swizzled [32][64] lo (Apply) or plain [64][32] mirror (Gram / Poly)
-  uint64_t* bar;   // this warp's load barrier
-  uint32_t phase;  // its parity
+struct EpiRing {
+  uint8_t* base;     // kEpiBufs buffers of kEpiChunkBytes (two halves each)
+  uint64_t* bar;     // kEpiBufs load barriers
+  uint32_t parity;   // bit i: parity of the next completion of bar[i]
+  uint32_t chunk;    // chunks handled so far by this warp (ring position)
 };
 
-// Bulk-load the chunk's inputs (lane 0 issues, every lane waits). False if the
-// wait gave up.
-__device__ __forceinline__ bool epi_load(const NsGemmParams& p, EpiCtx& e, const Tile& T,
-                                         const BankPlan& bp, int r0, int c0, int lane,
-                                         volatile int* abort_flag) {
-  if (T.phase == kGram) return true;
-  if (lane == 0) {
-    if (T.phase == kApply) {
-      const int y = T.mat * bp.Rp + r0;
-      mbar_arrive_expect_tx(e.bar, 2 * kEpiRows * kEpiCols * 2);
-      tma_load_2d(e.bufA, &p.maps[T.bank][kHiE0 + T.cur], e.bar, c0, y);
-      tma_load_2d(e.bufB, &p.maps[T.bank][kLoE], e.bar, c0, y);
-    } else {
-      mbar_arrive_expect_tx(e.bar, kEpiRows * kEpiCols * 2);
-      tma_load_2d(e.bufA, &p.maps[T.bank][kAE], e.bar, c0, T.mat * bp.rp + r0);
-    }
+__device__ __forceinline__ uint8_t* ring_buf(const EpiRing& e, uint32_t k) {
+  return e.base + (k % kEpiBufs) * kEpiChunkBytes;
+}
+
+// Lane 0 issues the bulk loads of ring chunk k (column c0 of this warp's rows).
+__device__ __forceinline__ void epi_issue_load(const NsGemmParams& p, const EpiRing& e,
+                                               const Tile& T, const BankPlan& bp, int r0, int c0,
+                                               uint32_t k) {
+  uint8_t* b = ring_buf(e, k);
+  uint64_t* bar = &e.bar[k % kEpiBufs];
+  if (T.phase == kApply) {
+    const int y = T.mat * bp.Rp + r0;
+    mbar_arrive_expect_tx(bar, kEpiChunkBytes);
+    tma_load_2d(b, &p.maps[T.bank][kHiE0 + T.cur], bar, c0, y);
+    tma_load_2d(b + kEpiHalfBytes, &p.maps[T.bank][kLoE], bar, c0, y);
+  } else if (T.phase == kPoly) {
+    mbar_arrive_expect_tx(bar, kEpiHalfBytes);
+    tma_load_2d(b, &p.maps[T.bank][kAE], bar, c0, T.mat * bp.rp + r0);
   }
-  const bool ok = mbar_wait(e.bar, e.phase, abort_flag, p.status, p.wait_limit_ns);
-  e.phase ^= 1u;
+}
+
+// Every lane waits for ring chunk k's loads. False if the wait gave up.
+__device__ __forceinline__ bool epi_wait_load(const NsGemmParams& p, EpiRing& e, uint32_t k,
+                                              volatile int* abort_flag) {
+  const uint32_t i = k % kEpiBufs;
+  const bool ok = mbar_wait(&e.bar[i], (e.parity >> i) & 1u, abort_flag, p.status, p.wait_limit_ns);
+  e.parity ^= 1u << i;
   return __all_sync(0xffffffffu, ok);
 }
 
-// Apply: x' = alpha x + beta D with x = hi + lo, for this lane's row of the chunk.
-__device__ __forceinline__ void epi_apply(const Tile& T, const BankPlan& bp, const EpiCtx& e,
-                                          int lane, const uint32_t (&r0)[32],
-                                          const uint32_t (&r1)[32]) {
+// Apply: x' = alpha x + beta D with x = hi + lo, for this lane's row.
+__device__ __forceinline__ void epi_apply(const Tile& T, const BankPlan& bp, uint8_t* buf, int lane,
+                                          const uint32_t (&r)[32]) {
   float alpha = T.a, beta = 1.0f;
   if (T.iter == 0) {  // the iterate holds U; X0 = s U
     const float s = bp.scale[T.mat];
@@ -235,50 +242,43 @@ __device__ __forceinline__ void epi_apply(const Tile& T, const BankPlan& bp, con
     beta = s;
   }
 #pragma unroll
-  for (int g = 0; g < 8; ++g) {
-    const uint32_t off = swz_off(lane, g);
-    const uint4 h4 = *reinterpret_cast<const uint4*>(e.bufA + off);
-    const uint4 l4 = *reinterpret_cast<const uint4*>(e.bufB + off);
+  for (int g = 0; g < 4; ++g) {
+    const uint32_t off = swz64_off(lane, g);
+    const uint4 h4 = *reinterpret_cast<const uint4*>(buf + off);
+    const uint4 l4 = *reinterpret_cast<const uint4*>(buf + kEpiHalfBytes + off);
     const uint32_t hw[4] = {h4.x, h4.y, h4.z, h4.w};
     const uint32_t lw[4] = {l4.x, l4.y, l4.z, l4.w};
     uint32_t ho[4], lo[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      const int c = 8 * g + 2 * h;
-      const float d0 = __uint_as_float(c < 32 ? r0[c & 31] : r1[c & 31]);
-      const float d1 = __uint_as_float(c + 1 < 32 ? r0[(c + 1) & 31] : r1[(c + 1) & 31]);
-      const float y0 = fmaf(alpha, bf16_lo_f(hw[h]) + bf16_lo_f(lw[h]), beta * d0);
-      const float y1 = fmaf(alpha, bf16_hi_f(hw[h]) + bf16_hi_f(lw[h]), beta * d1);
+      const float y0 = fmaf(alpha, bf16_lo_f(hw[h]) + bf16_lo_f(lw[h]), beta * __uint_as_float(r[8 * g + 2 * h]));
+      const float y1 = fmaf(alpha, bf16_hi_f(hw[h]) + bf16_hi_f(lw[h]), beta * __uint_as_float(r[8 * g + 2 * h + 1]));
       ho[h] = pack_bf16x2(y0, y1);
       lo[h] = pack_bf16x2(y0 - bf16_lo_f(ho[h]), y1 - bf16_hi_f(ho[h]));
     }
-    *reinterpret_cast<uint4*>(e.bufA + off) = make_uint4(ho[0], ho[1], ho[2], ho[3]);
-    *reinterpret_cast<uint4*>(e.bufB + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4*>(buf + off) = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+    *reinterpret_cast<uint4*>(buf + kEpiHalfBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
 // Gram (A = D, times s^2 at step 0) or Poly (B = b A + c D) for this lane's
-// row; the transposed copy goes to the mirror buffer when `mirror`.
-__device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, const EpiCtx& e,
-                                        int lane, bool mirror, const uint32_t (&r0)[32],
-                                        const uint32_t (&r1)[32]) {
+// row; the transposed copy goes to the mirror half when `mirror`.
+__device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, uint8_t* buf, int lane,
+                                        bool mirror, const uint32_t (&r)[32]) {
   float scl = 1.0f;
   if (T.phase == kGram && T.iter == 0) {  // the operand holds U; fold 1 / ||U||^2 in here
     const float s = bp.scale[T.mat];
     scl = s * s;
   }
-  unsigned short* mir = reinterpret_cast<unsigned short*>(e.bufB);
+  unsigned short* mir = reinterpret_cast<unsigned short*>(buf + kEpiHalfBytes);
 #pragma unroll
-  for (int g = 0; g < 8; ++g) {
-    const uint32_t off = swz_off(lane, g);
+  for (int g = 0; g < 4; ++g) {
+    const uint32_t off = swz64_off(lane, g);
     float v[8];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int c = 8 * g + t;
-      v[t] = __uint_as_float(c < 32 ? r0[c & 31] : r1[c & 31]);
-    }
+    for (int t = 0; t < 8; ++t) v[t] = __uint_as_float(r[8 * g + t]);
     if (T.phase == kPoly) {
-      const uint4 a4 = *reinterpret_cast<const uint4*>(e.bufA + off);
+      const uint4 a4 = *reinterpret_cast<const uint4*>(buf + off);
       const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
@@ -292,7 +292,7 @@ __device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, const
     uint32_t pk[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) pk[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
-    *reinterpret_cast<uint4*>(e.bufA + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4*>(buf + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     if (mirror) {
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
@@ -303,20 +303,22 @@ __device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, const
   }
 }
 
-// Bulk-store the chunk (lane 0, after every lane's writes are visible to TMA).
-__device__ __forceinline__ void epi_store(const NsGemmParams& p, const EpiCtx& e, const Tile& T,
-                                          const BankPlan& bp, int r0, int c0, int lane, bool mirror) {
+// Bulk-store ring chunk k (lane 0, after every lane's writes are visible to
+// the async proxy) as one bulk group.
+__device__ __forceinline__ void epi_store(const NsGemmParams& p, const Tile& T, const BankPlan& bp,
+                                          uint8_t* buf, int r0, int c0, int lane, bool mirror) {
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
     if (T.phase == kApply) {
       const int y = T.mat * bp.Rp + r0;
-      tma_store_2d(&p.maps[T.bank][kHiE0 + (T.cur ^ 1)], e.bufA, c0, y);
-      tma_store_2d(&p.maps[T.bank][kLoE], e.bufB, c0, y);
+      tma_store_2d(&p.maps[T.bank][kHiE0 + (T.cur ^ 1)], buf, c0, y);
+      tma_store_2d(&p.maps[T.bank][kLoE], buf + kEpiHalfBytes, c0, y);
     } else {
       const int base = T.mat * bp.rp;
-      tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAE : kBE], e.bufA, c0, base + r0);
-      if (mirror) tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAT : kBT], e.bufB, r0, base + c0);
+      tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAE : kBE], buf, c0, base + r0);
+      if (mirror)
+        tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAT : kBT], buf + kEpiHalfBytes, r0, base + c0);
     }
     bulk_commit();
   }
@@ -342,8 +344,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
-  uint64_t* epibar = done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + kEpiWarps);
+  uint64_t* epibar = done + 1;  // kEpiWarps x kEpiBufs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + kEpiWarps * kEpiBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -364,7 +366,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 2 * kEpiWarps);  // the leader's: both CTAs' epilogue warps
     }
     mbar_init(done, 1);
-    for (int w = 0; w < kEpiWarps; ++w) mbar_init(&epibar[w], 1);
+    for (int w = 0; w < kEpiWarps * kEpiBufs; ++w) mbar_init(&epibar[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -476,8 +478,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int ew = warp - 2;
-    EpiCtx e{epibuf + ew * kEpiBufBytes, epibuf + ew * kEpiBufBytes + kEpiBufBytes / 2, &epibar[ew], 0u};
+    EpiRing e{epibuf + ew * kEpiBufBytes, &epibar[ew * kEpiBufs], 0u, 0u};
     const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
+    constexpr int kChunks = 128 / kEpiCols;  // chunks per warp per tile
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -485,11 +488,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const Tile T = decode_tile(p, tile);
       const BankPlan& bp = p.bank[T.bank];
       const int r0 = T.m0 + kBM * static_cast<int>(rank) + 32 * q;  // first row of this warp
+      const int cw = T.n0 + half * 128;                              // first column of this warp
       const bool mirror = T.phase != kApply && T.n0 != T.m0;
-      // the epilogue's own TMA loads read the same finished phase
-      if (lane == 0 && T.phase != kGram &&
-          !wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit))
-        ok = false;
+      const bool loads = T.phase != kGram;
+      // the epilogue's own TMA loads read the same finished phase as the MMAs
+      if (lane == 0 && loads) {
+        if (!wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) ok = false;
+        else {
+          bulk_wait_read<1>();  // ring buffer of chunk e.chunk: its last store has read it
+          epi_issue_load(p, e, T, bp, r0, cw, e.chunk);
+        }
+      }
       if (!__all_sync(0xffffffffu, ok)) break;
       // the tcgen05.ld below is warp-collective: leave only if the whole warp does
       const bool got = mbar_wait_cluster(&tfull[acc], acc_phase, abort_flag, p.status, limit);
@@ -498,20 +507,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                           static_cast<uint32_t>(acc * kBN + half * 128);
 #pragma unroll 1
-      for (int jj = 0; jj < 2; ++jj) {
-        const int c0 = T.n0 + half * 128 + jj * kEpiCols;
-        if (lane == 0) bulk_wait_read();  // the buffers' previous stores have read them
+      for (int j = 0; j < kChunks; ++j) {
+        const uint32_t k = e.chunk;
+        const int c0 = cw + j * kEpiCols;
+        if (lane == 0) {
+          if (loads && j + 1 < kChunks) {
+            bulk_wait_read<1>();  // buffer of chunk k+1 was last stored from by chunk k-2
+            epi_issue_load(p, e, T, bp, r0, c0 + kEpiCols, k + 1);
+          } else if (!loads) {
+            bulk_wait_read<kEpiBufs - 1>();  // buffer of chunk k was last stored from by chunk k-3
+          }
+        }
         __syncwarp();
-        if (!epi_load(p, e, T, bp, r0, c0, lane, abort_flag)) { ok = false; break; }
-        uint32_t ra[32], rb[32];
-        tmem_ld32(tb + jj * kEpiCols, ra);
-        tmem_ld32(tb + jj * kEpiCols + 32, rb);
+        uint32_t r[32];
+        tmem_ld32(tb + j * kEpiCols, r);
+        if (loads && !epi_wait_load(p, e, k, abort_flag)) {
+          tmem_ld_wait();
+          ok = false;
+          break;
+        }
         tmem_ld_wait();
+        uint8_t* buf = ring_buf(e, k);
         if (T.phase == kApply)
-          epi_apply(T, bp, e, lane, ra, rb);
+          epi_apply(T, bp, buf, lane, r);
         else
-          epi_sym(T, bp, e, lane, mirror, ra, rb);
-        epi_store(p, e, T, bp, r0, c0, lane, mirror);
+          epi_sym(T, bp, buf, lane, mirror, r);
+        epi_store(p, T, bp, buf, r0, c0, lane, mirror);
+        e.chunk = k + 1;
       }
       if (!ok) break;
       tc_fence_before();

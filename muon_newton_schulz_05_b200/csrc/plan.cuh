@@ -22,15 +22,18 @@ constexpr int kTile = 256;         // GEMM tile (rows and cols) computed by one 
 constexpr int kBM = 128;           // tile rows held by one CTA of the pair
 constexpr int kBN = 256;           // tile cols (UMMA N); each CTA loads kBN/2 of B
 constexpr int kBK = 64;            // K per pipeline stage (one 128-byte swizzle row)
-constexpr int kStages = 5;         // TMA -> MMA pipeline depth
+constexpr int kStages = 4;         // TMA -> MMA pipeline depth (4..7 measured equal)
 constexpr int kATileBytes = kBM * kBK * 2;
 constexpr int kBTileBytes = (kBN / 2) * kBK * 2;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kEpiWarps = 8;       // two per TMEM lane quadrant
-constexpr int kEpiRows = 32;       // epilogue chunk: 32 rows x 64 columns per warp
-constexpr int kEpiCols = 64;
-constexpr int kEpiBufBytes = 2 * kEpiRows * kEpiCols * 2;  // two bf16 chunk buffers per warp
-constexpr int kGemmSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 1024 + 256;
+constexpr int kEpiRows = 32;       // epilogue chunk: 32 rows x 32 columns per warp
+constexpr int kEpiCols = 32;
+constexpr int kEpiHalfBytes = kEpiRows * kEpiCols * 2;      // one bf16 chunk
+constexpr int kEpiChunkBytes = 2 * kEpiHalfBytes;           // hi + lo, or out + mirror
+constexpr int kEpiBufs = 3;                                 // ring of chunk buffers per warp
+constexpr int kEpiBufBytes = kEpiBufs * kEpiChunkBytes;
+constexpr int kGemmSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 1024 + 512;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, then epilogue
 constexpr int kChunk = 8192;       // padded elements per block in the momentum pass
 constexpr int kMaxMaps = 13;
@@ -38,9 +41,9 @@ constexpr int kMaxMaps = 13;
 enum Phase : int { kGram = 0, kPoly = 1, kApply = 2 };
 
 // Tensor-map slots per bank. Operand maps (128-byte swizzle): K-major boxes
-// of 128 rows x 64 columns, MN-major boxes of 64 x 64. Epilogue maps: 32 rows
-// x 64 columns with 128-byte swizzle (row-wise chunks), and 64 rows x 32
-// columns unswizzled (transposed mirror chunks of A and B).
+// of 128 rows x 64 columns, MN-major boxes of 64 x 64. Epilogue maps: 32 x 32
+// chunks, 64-byte swizzle for row-wise chunks, unswizzled for the transposed
+// mirror chunks of A and B.
 enum MapSlot : int {
   kHiK0 = 0, kHiK1 = 1, kHiMN0 = 2, kHiMN1 = 3, kAK = 4, kBK_ = 5,
   kHiE0 = 6, kHiE1 = 7, kLoE = 8, kAE = 9, kAT = 10, kBE = 11, kBT = 12

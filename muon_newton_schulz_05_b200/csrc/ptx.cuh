@@ -100,10 +100,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
-// Wait until every committed bulk store of this thread has finished reading
-// shared memory (the buffer may be reused).
+// Wait until at most N of this thread's most recent committed bulk stores are
+// still reading shared memory (the older ones' buffers may be reused).
+template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
 // Wait until every committed bulk store of this thread is complete.
