@@ -282,6 +282,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   }
   if (ev_before && cudaEventRecord(ev_before, stream) != cudaSuccess) return MUON_ERR_CUDA;
   gp.ns_steps = hp->ns_steps;
+  gp.keep_lo = v == Variant::kOrtho ? 1 : 0;
   for (int i = 0; i < 3 * hp->ns_steps; ++i) gp.coef[i] = hp->coeffs[i];
   int sym = 0, app = 0;
   for (int b = 0; b < nbanks; ++b) {
@@ -301,6 +302,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   up.nbanks = nbanks;
   up.mode = v == Variant::kMuon ? kUpdDecoupled : (v == Variant::kAnvil ? kUpdCautious : kUpdWriteO);
   up.final_buf = hp->ns_steps & 1;
+  up.use_lo = v == Variant::kOrtho ? 1 : 0;
   up.lr_wd = hp->lr * hp->weight_decay;
   up.ema_beta = hp->ema_beta;
   long long total = 0;

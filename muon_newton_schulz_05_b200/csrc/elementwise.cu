@@ -225,9 +225,14 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
         const long long off = mat * padded + row * bp.Cp + col;
         float o[8], h8[8], l8[8];
         load8(hi, MUON_BF16, off, h8);
-        load8(lo, MUON_BF16, off, l8);
+        if (p.use_lo) {
+          load8(lo, MUON_BF16, off, l8);
 #pragma unroll
-        for (int t = 0; t < 8; ++t) o[t] = h8[t] + l8[t];
+          for (int t = 0; t < 8; ++t) o[t] = h8[t] + l8[t];
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) o[t] = h8[t];
+        }
         if (p.mode == kUpdWriteO) {
           store8(io.param, io.param_dtype, e, o);
           continue;
@@ -254,7 +259,7 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
         const long long row = rem / bp.C;
         const long long col = rem - row * bp.C;
         const long long off = mat * padded + row * bp.Cp + col;
-        const float o = __bfloat162float(hi[off]) + __bfloat162float(lo[off]);
+        const float o = __bfloat162float(hi[off]) + (p.use_lo ? __bfloat162float(lo[off]) : 0.0f);
         if (p.mode == kUpdWriteO) {
           round_store1(io.param, io.param_dtype, e, o);
           continue;

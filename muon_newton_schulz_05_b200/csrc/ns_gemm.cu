@@ -313,7 +313,10 @@ __device__ __forceinline__ void epi_store(const NsGemmParams& p, const Tile& T, 
     if (T.phase == kApply) {
       const int y = T.mat * bp.Rp + r0;
       tma_store_2d(&p.maps[T.bank][kHiE0 + (T.cur ^ 1)], buf, c0, y);
-      tma_store_2d(&p.maps[T.bank][kLoE], buf + kEpiHalfBytes, c0, y);
+      // the parameter update takes O in bf16; the low part of the last
+      // iterate is stored only when O itself is the requested output
+      if (T.iter + 1 < p.ns_steps || p.keep_lo)
+        tma_store_2d(&p.maps[T.bank][kLoE], buf + kEpiHalfBytes, c0, y);
     } else {
       const int base = T.mat * bp.rp;
       tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAE : kBE], buf, c0, base + r0);

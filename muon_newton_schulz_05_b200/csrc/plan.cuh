@@ -78,6 +78,7 @@ struct NsGemmParams {
   int apply_begin[MUON_MAX_BANKS + 1];  // prefix sums of count * tiles_apply
   int nbanks;
   int ns_steps;
+  int keep_lo;                          // last step also stores lo (full-precision O)
   float coef[3 * MUON_MAX_NS_STEPS];    // (a, b, c) per step
   int* status;                          // device status word
   unsigned long long wait_limit_ns;
@@ -125,6 +126,7 @@ struct UpdParams {
   int nbanks;
   int mode;
   int final_buf;        // hi buffer holding the last iterate
+  int use_lo;           // O = hi + lo (else the bf16 hi alone)
   float lr_wd;          // lr * weight_decay
   float ema_beta;
 };
