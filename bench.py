@@ -30,7 +30,13 @@ sys.path.insert(0, ROOT)
 METRIC = "Muon steps/s on GPT-124M matrix bank; NS TFLOP/s as % bf16 tensor peak"
 UNIT = "steps/s"
 WORKLOAD_ID = 2
-LAUNCHES_PER_STEP_FIXED = 3  # momentum+norm, norm finalize, update
+# kernel launches per step: momentum+norm, norm finalize, the Newton-Schulz
+# chain (one persistent launch), update
+LAUNCHES_PER_STEP = 4
+# DRAM bytes (read + write) of one Newton-Schulz chain launch on this workload,
+# from the ncu capture summarised in profiles/ns_gemm_gpt124m_bank.md. Set to
+# None whenever ns_gemm_kernel changes until it is captured again.
+NS_CHAIN_DRAM_BYTES = 5.815693e9
 
 
 def _args():
@@ -83,6 +89,23 @@ def _config(w, extra=None):
     if extra:
         c.update(extra)
     return c
+
+
+# --------------------------------------------------------------- multi-rank
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """The largest value of x over all ranks (x itself without a process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, max_ms: float) -> float:
+    """Whole-job steps/s: every rank stepped its own bank `steps` times and the
+    slowest rank took max_ms."""
+    return world * steps / (max_ms / 1e3)
 
 
 # --------------------------------------------------------------- CPU oracle
@@ -234,8 +257,7 @@ def run_native(args):
     H = mb.Hparams.from_dict(w.hp)
     stream = torch.cuda.current_stream(dev)
     flops_step = _ns_flops(w)
-    k = len(w.hp["coeffs"])
-    launches_per_step = LAUNCHES_PER_STEP_FIXED + 3 * k
+    launches_per_step = LAUNCHES_PER_STEP
 
     for _ in range(args.warmup):
         mb.muon_step(banks, H, ws)
@@ -271,12 +293,9 @@ def run_native(args):
     pre_ms = [ev[4 * s].elapsed_time(ev[4 * s + 1]) for s in range(K)]
     post_ms = [ev[4 * s + 2].elapsed_time(ev[4 * s + 3]) for s in range(K)]
     assert mb.device_status(ws) == 0
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist if world > 1 else None, dev)
     ms_per_step = total_ms / K
-    value = world * K / (total_ms / 1e3)
+    value = job_throughput(world, K, total_ms)
 
     ns_avg_ms = statistics.mean(ns_ms)
     achieved = flops_step / (ns_avg_ms * 1e-3) / 1e12
@@ -305,12 +324,8 @@ def run_native(args):
                 hp_.copy_(bk.param, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+        e2e = {"value": job_throughput(world, E, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
                "what": "per step: pinned host->device copy of the bf16 gradients, muon_step, "
                        "device->host copy of the updated bf16 parameters"}
@@ -334,8 +349,11 @@ def run_native(args):
         "config": _config(w),
         "roofline": {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": None,
-            "kernel": "ns_gemm_kernel (the 15 launches of one Newton-Schulz chain)",
+            "frac": achieved / peak, "traffic": NS_CHAIN_DRAM_BYTES,
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
+                              "(profiles/ns_gemm_gpt124m_bank.md)",
+            "kernel": "ns_gemm_kernel (one persistent launch: 5 Newton-Schulz steps x "
+                      "Gram/Poly/Apply over the 72-matrix bank)",
             "flops_per_launch": flops_step, "launch_ms": ns_avg_ms,
             "peak_kind": f"bf16 dense sustained, {peaks['src']}",
             "frac_of_burst": achieved / peaks["burst"],
