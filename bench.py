@@ -47,6 +47,9 @@ def _args():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
+                    help="1..5 (default 2, the GPT-124M bank the metric names); the others "
+                         "are measured for documentation only")
     return ap.parse_args()
 
 
@@ -60,9 +63,9 @@ def _peaks():
         return dict(hbm=6650.0, burst=1590.0, sustained=1400.0, src="fallback")
 
 
-def _workload():
+def _workload(wid: int = WORKLOAD_ID):
     import muon_inputs as mi
-    return mi.workloads()[WORKLOAD_ID]
+    return mi.workloads()[wid]
 
 
 def _ns_flops(w) -> float:
@@ -78,13 +81,22 @@ def _ns_flops(w) -> float:
 
 
 def _config(w, extra=None):
-    c = {"workload": "gpt124m_matrix_bank",
+    names = {1: "single_256x512_fp32", 2: "gpt124m_matrix_bank", 3: "square_1024x1024x64_bank",
+             4: "transformer_2p5b_matrix_bank", 5: "anvil_gpt124m_bank_plus_readout"}
+    if w.variant == "anvil":
+        mom = (f"fp32 fast/slow, beta {w.hp['beta_fast']}/{w.hp['beta_slow']}, cautious decay, "
+               f"EMA {w.hp['ema_beta']}")
+    else:
+        mom = f"fp32, mu={w.hp['mu']}" + (", nesterov" if w.hp.get("nesterov") else "")
+    touched = w.n_params * (2 + 2 + 8 + 6) / 1e9
+    c = {"workload": names.get(w.cid, w.name),
          "banks": [f"{b.count}x{b.rows}x{b.cols}" for b in w.banks],
          "params": w.n_params, "param_dtype": w.param_dtype, "grad_dtype": w.grad_dtype,
-         "momentum": "fp32, mu=0.95, nesterov", "ns_steps": len(w.hp["coeffs"]),
+         "momentum": mom, "ns_steps": len(w.hp["coeffs"]),
          "coeffs": list(w.hp["coeffs"][0]), "lr": w.hp["lr"], "weight_decay": w.hp["weight_decay"],
-         "grads": "N(0,1e-3^2) + rank-4 spike at 10x RMS",
-         "l2": "inputs larger than L2: ~1.2 GB touched per step (126 MB L2), no flush",
+         "grads": f"N(0,{w.grad_sigma:g}^2)" + (f" + rank-{w.spike_rank} spike at 10x RMS" if w.spike_rank else ""),
+         "l2": (f"inputs larger than L2: ~{touched:.2f} GB touched per step (126 MB L2), no flush"
+                if touched > 0.126 else f"~{touched*1e3:.0f} MB touched per step: fits in L2, no flush"),
          "parallelism": "replica per GPU (independent banks)"}
     if extra:
         c.update(extra)
@@ -121,7 +133,7 @@ def _cpu_threads():
     return len(os.sched_getaffinity(0))
 
 
-def _oracle_sample_time(w, budget_s: float, start_step: int = 0):
+def _oracle_sample_time(w, budget_s: float, start_step: int = 0, max_per_shape: int = 12):
     """Oracle Muon step on matrices of the bank, cycling the three shapes,
     until budget_s of CPU work; returns (seconds per full-bank step, sample
     description)."""
@@ -138,14 +150,17 @@ def _oracle_sample_time(w, budget_s: float, start_step: int = 0):
             g = oracle.as_f64(mi.make_grads(w, b, start_step, [i])[0])
             m = np.zeros_like(g)
             t0 = time.perf_counter()
-            oracle.muon_step(th, g, m, w.hp, w.param_dtype)
+            if w.variant == "anvil":
+                oracle.anvil_step(th, g, m, m, w.hp, w.param_dtype)
+            else:
+                oracle.muon_step(th, g, m, w.hp, w.param_dtype)
             per_shape[b].append(time.perf_counter() - t0)
         idx += 1
-        if time.perf_counter() - t_start >= budget_s or idx >= 12:
+        if time.perf_counter() - t_start >= budget_s or idx >= max(1, min(12, max_per_shape)):
             break
     full = sum(w.banks[b].count * statistics.mean(ts) for b, ts in per_shape.items())
     n = sum(len(ts) for ts in per_shape.values())
-    desc = (f"oracle muon_step (float64, numpy) on {n} matrices ({idx} of each shape "
+    desc = (f"oracle {w.variant}_step (float64, numpy) on {n} matrices ({idx} of each shape "
             f"{', '.join(f'{s.rows}x{s.cols}' for s in w.banks)}), mean time per shape "
             f"scaled by the bank's counts {[s.count for s in w.banks]}")
     return full, desc
@@ -155,7 +170,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = _workload()
+    w = _workload(args.workload)
     for _ in range(args.warmup):
         _oracle_sample_time(w, 0.0)
     times = []
@@ -243,8 +258,9 @@ def run_native(args):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = _workload()
+    w = _workload(args.workload)
     peaks = _peaks()
+    anvil = w.variant == "anvil"
 
     # -------- inputs (host-generated, seeded, uploaded before timing)
     banks, host_grads = [], []
@@ -252,15 +268,20 @@ def run_native(args):
         th = mi.make_params(w, b).to(dev)
         g = mi.make_grads(w, b, 0)
         host_grads.append(g.pin_memory())
-        banks.append(mb.Bank(th, g.to(dev), torch.zeros(th.shape, dtype=torch.float32, device=dev)))
+        z = torch.zeros(th.shape, dtype=torch.float32, device=dev)
+        if anvil:
+            banks.append(mb.Bank(th, g.to(dev), z, torch.zeros_like(z), th.float()))
+        else:
+            banks.append(mb.Bank(th, g.to(dev), z))
     ws = mb.alloc_workspace([bk.shape for bk in banks], device=dev)
     H = mb.Hparams.from_dict(w.hp)
+    step_fn = mb.anvil_step if anvil else mb.muon_step
     stream = torch.cuda.current_stream(dev)
     flops_step = _ns_flops(w)
     launches_per_step = LAUNCHES_PER_STEP
 
     for _ in range(args.warmup):
-        mb.muon_step(banks, H, ws)
+        step_fn(banks, H, ws)
     torch.cuda.synchronize()
     assert mb.device_status(ws) == 0
 
@@ -281,7 +302,7 @@ def run_native(args):
         e_step0, e_ns0, e_ns1, e_step1 = ev[4 * s:4 * s + 4]
         e_step0.record(stream)
         mb.set_ns_events(e_ns0, e_ns1)
-        mb.muon_step(banks, H, ws)
+        step_fn(banks, H, ws)
         e_step1.record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -301,10 +322,14 @@ def run_native(args):
     achieved = flops_step / (ns_avg_ms * 1e-3) / 1e12
     elem_bytes = sum(b.count * b.rows * b.cols for b in w.banks)
     # algorithmic bytes of the two elementwise passes per element:
-    # momentum+norm: G bf16 read 2, M read+write 8, iterate hi+lo write 4 = 14
-    # update: iterate hi+lo read 4, theta bf16 read+write 4 = 8
-    pre_gbs = elem_bytes * 14 / (statistics.mean(pre_ms) * 1e-3) / 1e9
-    post_gbs = elem_bytes * 8 / (statistics.mean(post_ms) * 1e-3) / 1e9
+    # momentum+norm: G read, M read+write 8 (ANVIL: both momenta 16), iterate hi+lo write 4
+    # update: O (bf16 hi) read 2, theta read+write (ANVIL: + slow momentum 4, EMA r+w 8)
+    gsz = 2 if w.grad_dtype == "bf16" else 4
+    psz = 2 if w.param_dtype == "bf16" else 4
+    pre_b = gsz + (16 if anvil else 8) + 4
+    post_b = 2 + 2 * psz + (12 if anvil else 0)
+    pre_gbs = elem_bytes * pre_b / (statistics.mean(pre_ms) * 1e-3) / 1e9
+    post_gbs = elem_bytes * post_b / (statistics.mean(post_ms) * 1e-3) / 1e9
 
     # -------- end to end through the public API with host buffers
     e2e = None
@@ -319,7 +344,7 @@ def run_native(args):
         for s in range(E):
             for bk, g in zip(banks, host_grads):
                 bk.grad.copy_(g, non_blocking=True)
-            mb.muon_step(banks, H, ws)
+            step_fn(banks, H, ws)
             for bk, hp_ in zip(banks, host_params):
                 hp_.copy_(bk.param, non_blocking=True)
         e1.record(stream)
@@ -349,7 +374,8 @@ def run_native(args):
         "config": _config(w),
         "roofline": {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": NS_CHAIN_DRAM_BYTES,
+            "frac": achieved / peak,
+            "traffic": NS_CHAIN_DRAM_BYTES if args.workload == WORKLOAD_ID else None,
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
                               "(profiles/ns_gemm_gpt124m_bank.md)",
             "kernel": "ns_gemm_kernel (one persistent launch: 5 Newton-Schulz steps x "
