@@ -149,13 +149,29 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
     const int nb = p.rp / kTile;
     p.tiles_sym = nb * (nb + 1) / 2;
     p.tiles_apply = (p.Rp / kTile) * (p.Cp / kTile);
+    // Split the Gram product along K when the bank has too few Gram tiles to
+    // spread and K is much longer than the Gram is wide (e.g. a 768 x 50304
+    // readout: 6 tiles of 788 K blocks). Splits keep >= 32 K blocks each.
+    const int kg = (p.tall ? p.Rp : p.Cp) / kBK;
+    p.ksplit = 1;
+    if (p.count * p.tiles_sym < 48 && kg * kBK >= 8 * p.rp) {
+      p.ksplit = kg / 32;
+      if (p.ksplit > kMaxSplit) p.ksplit = kMaxSplit;
+      if (p.ksplit < 1) p.ksplit = 1;
+    }
+    p.kc = (kg + p.ksplit - 1) / p.ksplit;
+    if (p.ksplit > 1) p.ksplit = (kg + p.kc - 1) / p.kc;  // no empty split
+    p.tiles_red = p.ksplit > 1 ? p.tiles_sym * kRedSub : 0;
     const size_t it_bytes = static_cast<size_t>(p.count) * padded * 2;
     const size_t sq_bytes = static_cast<size_t>(p.count) * p.rp * p.rp * 2;
     const size_t o_hi0 = take(it_bytes), o_hi1 = take(it_bytes), o_lo = take(it_bytes);
     const size_t o_A = take(sq_bytes), o_B = take(sq_bytes);
     const size_t o_part = take(static_cast<size_t>(p.count) * p.chunks * 4);
     const size_t o_scale = take(static_cast<size_t>(p.count) * 4);
-    const size_t o_cnt = take(static_cast<size_t>(p.count) * 3 * 4);
+    const size_t o_cnt = take(static_cast<size_t>(p.count) * 4 * 4);
+    const size_t o_gpart = p.ksplit > 1 ? take(static_cast<size_t>(p.count) * p.tiles_sym * p.ksplit *
+                                              kTile * kTile * 4)
+                                       : 0;
     if (base) {
       p.hi[0] = reinterpret_cast<__nv_bfloat16*>(base + o_hi0);
       p.hi[1] = reinterpret_cast<__nv_bfloat16*>(base + o_hi1);
@@ -165,6 +181,7 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
       p.partial = reinterpret_cast<float*>(base + o_part);
       p.scale = reinterpret_cast<float*>(base + o_scale);
       p.counters = reinterpret_cast<int*>(base + o_cnt);
+      p.part = p.ksplit > 1 ? reinterpret_cast<float*>(base + o_gpart) : nullptr;
       plans[b] = p;
     }
   }
@@ -172,12 +189,13 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
 }
 
 muon_status encode_map(CUtensorMap* m, void* ptr, int64_t inner, int64_t outer, int box_inner,
-                       int box_outer, CUtensorMapSwizzle swz) {
+                       int box_outer, CUtensorMapSwizzle swz, bool fp32 = false) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * 2};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * (fp32 ? 4 : 2)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+  CUresult r = g_encode(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        2, ptr, dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MUON_OK : MUON_ERR_CUDA;
@@ -209,6 +227,10 @@ muon_status encode_bank_maps(const BankPlan& p, CUtensorMap* maps) {
   for (const Spec& sp : specs) {
     muon_status st = encode_map(&maps[sp.slot], sp.ptr, sp.inner, sp.outer, sp.bi, sp.bo, sp.swz);
     if (st != MUON_OK) return st;
+  }
+  if (p.ksplit > 1) {
+    const int64_t prow = static_cast<int64_t>(p.count) * p.tiles_sym * p.ksplit * kTile;
+    return encode_map(&maps[kPartE], p.part, kTile, prow, kEpiCols, kEpiRows, sw, true);
   }
   return MUON_OK;
 }
@@ -284,13 +306,19 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   gp.ns_steps = hp->ns_steps;
   gp.keep_lo = v == Variant::kOrtho ? 1 : 0;
   for (int i = 0; i < 3 * hp->ns_steps; ++i) gp.coef[i] = hp->coeffs[i];
-  int sym = 0, app = 0;
+  int gram = 0, red = 0, sym = 0, app = 0;
   for (int b = 0; b < nbanks; ++b) {
+    gp.gram_begin[b] = gram;
+    gp.red_begin[b] = red;
     gp.sym_begin[b] = sym;
     gp.apply_begin[b] = app;
+    gram += plans[b].count * plans[b].tiles_sym * plans[b].ksplit;
+    red += plans[b].count * plans[b].tiles_red;
     sym += plans[b].count * plans[b].tiles_sym;
     app += plans[b].count * plans[b].tiles_apply;
   }
+  gp.gram_begin[nbanks] = gram;
+  gp.red_begin[nbanks] = red;
   gp.sym_begin[nbanks] = sym;
   gp.apply_begin[nbanks] = app;
   if (launch_ns_gemm(gp, sms, stream) != cudaSuccess) return MUON_ERR_CUDA;

@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(128) norm_finalize_kernel(const __grid_constan
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) bp.scale[mat] = static_cast<float>(1.0 / (sqrt(s) + static_cast<double>(p.eps)));
   // the Newton-Schulz chain's per-matrix completion counters start at zero
-  if (lane < 3) bp.counters[3 * mat + lane] = 0;
+  if (lane < 4) bp.counters[4 * mat + lane] = 0;
 }
 
 cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total_mats,

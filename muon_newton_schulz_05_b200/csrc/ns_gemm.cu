@@ -33,6 +33,8 @@ namespace muon {
 
 struct Tile {
   int bank, mat, m0, n0, nkb;
+  int kb0;                    // first 64-deep K block (split Gram tiles)
+  int sym_t, split, sub;      // symmetric tile index, K split, reduce sub-tile
   int phase, iter, cur;       // Phase, Newton-Schulz step, hi buffer holding X_iter
   float a, b, c;              // this step's coefficients
   int a_map, a_mn, a_base;
@@ -54,23 +56,32 @@ __device__ __forceinline__ void sym_tile(int t, int nb, int& i, int& j) {
   j = ii + t;
 }
 
+__host__ __device__ __forceinline__ int tiles_per_step(const NsGemmParams& p) {
+  return p.gram_begin[p.nbanks] + p.red_begin[p.nbanks] + p.sym_begin[p.nbanks] +
+         p.apply_begin[p.nbanks];
+}
+
 __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   Tile T;
-  const int S = p.sym_begin[p.nbanks];
-  const int per_iter = 2 * S + p.apply_begin[p.nbanks];
+  const int G = p.gram_begin[p.nbanks], Rd = p.red_begin[p.nbanks], S = p.sym_begin[p.nbanks];
+  const int per_iter = tiles_per_step(p);
   T.iter = tile / per_iter;
   int r = tile - T.iter * per_iter;
   const int* begin;
-  if (r < S) {
+  if (r < G) {
     T.phase = kGram;
-    begin = p.sym_begin;
-  } else if (r < 2 * S) {
+    begin = p.gram_begin;
+  } else if (r < G + Rd) {
+    T.phase = kReduce;
+    r -= G;
+    begin = p.red_begin;
+  } else if (r < G + Rd + S) {
     T.phase = kPoly;
-    r -= S;
+    r -= G + Rd;
     begin = p.sym_begin;
   } else {
     T.phase = kApply;
-    r -= 2 * S;
+    r -= G + Rd + S;
     begin = p.apply_begin;
   }
   int b = 0;
@@ -82,6 +93,10 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   T.a = p.coef[3 * T.iter];
   T.b = p.coef[3 * T.iter + 1];
   T.c = p.coef[3 * T.iter + 2];
+  T.kb0 = 0;
+  T.split = 0;
+  T.sub = 0;
+  T.sym_t = 0;
   if (T.phase == kApply) {
     T.mat = local / bp.tiles_apply;
     const int t = local - T.mat * bp.tiles_apply;
@@ -89,22 +104,50 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
     T.m0 = (t / nbn) * kTile;
     T.n0 = (t % nbn) * kTile;
   } else {
-    T.mat = local / bp.tiles_sym;
-    const int t = local - T.mat * bp.tiles_sym;
+    int t;
+    if (T.phase == kGram) {
+      const int per = bp.tiles_sym * bp.ksplit;
+      T.mat = local / per;
+      const int t2 = local - T.mat * per;
+      t = t2 / bp.ksplit;
+      T.split = t2 - t * bp.ksplit;
+    } else if (T.phase == kReduce) {
+      T.mat = local / bp.tiles_red;
+      const int t3 = local - T.mat * bp.tiles_red;
+      t = t3 / kRedSub;
+      T.sub = t3 - t * kRedSub;
+    } else {
+      T.mat = local / bp.tiles_sym;
+      t = local - T.mat * bp.tiles_sym;
+    }
+    T.sym_t = t;
     int i, j;
     sym_tile(t, bp.rp / kTile, i, j);
     T.m0 = i * kTile;
     T.n0 = j * kTile;
   }
-  // Gram(k) reads X_k (all of Apply(k-1)); Poly(k) reads A (all of Gram(k));
-  // Apply(k) reads B (all of Poly(k)). Earlier phases are implied by these.
-  int* cnt = bp.counters + 3 * T.mat;
+  // Gram(k) reads X_k (all of Apply(k-1)); Reduce(k) sums all of Gram(k)'s
+  // partials; Poly(k) reads A (all of Reduce(k), or of Gram(k) when the bank
+  // is not split); Apply(k) reads B (all of Poly(k)). Earlier phases are
+  // implied by these.
+  int* cnt = bp.counters + 4 * T.mat;
   T.done_cnt = cnt + T.phase;
   if (T.phase == kGram) {
     T.dep_cnt = cnt + kApply;
     T.dep_target = kTileParts * bp.tiles_apply * T.iter;
+  } else if (T.phase == kReduce) {
+    T.dep_cnt = cnt + kGram;
+    T.dep_target = kTileParts * bp.tiles_sym * bp.ksplit * (T.iter + 1);
+  } else if (T.phase == kPoly) {
+    if (bp.ksplit > 1) {
+      T.dep_cnt = cnt + kReduce;
+      T.dep_target = kTileParts * bp.tiles_red * (T.iter + 1);
+    } else {
+      T.dep_cnt = cnt + kGram;
+      T.dep_target = kTileParts * bp.tiles_sym * (T.iter + 1);
+    }
   } else {
-    T.dep_cnt = cnt + (T.phase - 1);
+    T.dep_cnt = cnt + kPoly;
     T.dep_target = kTileParts * bp.tiles_sym * (T.iter + 1);
   }
   const int cur = T.cur;
@@ -120,6 +163,15 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
       T.b_map = kHiMN0 + cur; T.b_mn = 1; T.b_base = xbase;
       T.nkb = bp.Rp / kBK;
     }
+    if (bp.ksplit > 1) {  // this split's K blocks
+      T.kb0 = T.split * bp.kc;
+      T.nkb = min(bp.kc, T.nkb - T.kb0);
+    }
+  } else if (T.phase == kReduce) {
+    T.nkb = 0;
+    T.a_map = T.b_map = 0;
+    T.a_mn = T.b_mn = 0;
+    T.a_base = T.b_base = 0;
   } else if (T.phase == kPoly) {  // D[m][n] = sum_k A[m][k] A[n][k]
     T.a_map = kAK; T.a_mn = 0; T.a_base = sbase;
     T.b_map = kAK; T.b_mn = 0; T.b_base = sbase;
@@ -266,7 +318,7 @@ __device__ __forceinline__ void epi_apply(const Tile& T, const BankPlan& bp, uin
 __device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, uint8_t* buf, int lane,
                                         bool mirror, const uint32_t (&r)[32]) {
   float scl = 1.0f;
-  if (T.phase == kGram && T.iter == 0) {  // the operand holds U; fold 1 / ||U||^2 in here
+  if (T.phase != kPoly && T.iter == 0) {  // Gram / Reduce of U: fold 1 / ||U||^2 in here
     const float s = bp.scale[T.mat];
     scl = s * s;
   }
@@ -319,12 +371,93 @@ __device__ __forceinline__ void epi_store(const NsGemmParams& p, const Tile& T, 
         tma_store_2d(&p.maps[T.bank][kLoE], buf + kEpiHalfBytes, c0, y);
     } else {
       const int base = T.mat * bp.rp;
-      tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAE : kBE], buf, c0, base + r0);
+      tma_store_2d(&p.maps[T.bank][T.phase == kPoly ? kBE : kAE], buf, c0, base + r0);
       if (mirror)
-        tma_store_2d(&p.maps[T.bank][T.phase == kGram ? kAT : kBT], buf + kEpiHalfBytes, r0, base + c0);
+        tma_store_2d(&p.maps[T.bank][T.phase == kPoly ? kBT : kAT], buf + kEpiHalfBytes, r0, base + c0);
     }
     bulk_commit();
   }
+}
+
+// ------------------------------------------------- split Gram: partials, Reduce
+// fp32 chunk buffers use the 128-byte swizzle of a 32 x 32 fp32 box: 16-byte
+// group g of row r at r*128 + ((g ^ (r & 7)) * 16).
+__device__ __forceinline__ uint32_t swz128_off(int r, int g) {
+  return static_cast<uint32_t>(r * 128 + ((g ^ (r & 7)) << 4));
+}
+
+// Split Gram tile: this lane's row of the fp32 partial chunk goes to the
+// buffer, then the chunk is bulk-stored at (pcol, prow) of the partial map.
+__device__ __forceinline__ void epi_partial(const NsGemmParams& p, const Tile& T, uint8_t* buf,
+                                            int lane, int prow, int pcol, const uint32_t (&r)[32]) {
+#pragma unroll
+  for (int g = 0; g < 8; ++g)
+    *reinterpret_cast<uint4*>(buf + swz128_off(lane, g)) =
+        make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(&p.maps[T.bank][kPartE], buf, pcol, prow);
+    bulk_commit();
+  }
+}
+
+// Reduce sub-tile: this warp sums the ksplit partials of its 32 x 32 chunk in
+// split order (deterministic), folds in 1/||U||^2 at step 0, and stores the
+// bf16 chunk of A and, off the diagonal, its mirror. Requires every earlier
+// bulk store of the warp to be complete (all ring buffers free). False if a
+// wait gave up.
+__device__ __forceinline__ bool epi_reduce(const NsGemmParams& p, EpiRing& e, const Tile& T,
+                                           const BankPlan& bp, int lane, int rank, int q, int half,
+                                           volatile int* abort_flag) {
+  const int ks = bp.ksplit;
+  const int prow0 = (T.mat * bp.tiles_sym + T.sym_t) * ks * kTile + kBM * rank + 32 * q;
+  const int pcol = half * 128 + kEpiCols * T.sub;
+  const CUtensorMap* pmap = &p.maps[T.bank][kPartE];
+  if (lane == 0) {
+    for (int s = 0; s < 2 && s < ks; ++s) {
+      mbar_arrive_expect_tx(&e.bar[s], kEpiChunkBytes);
+      tma_load_2d(e.base + s * kEpiChunkBytes, pmap, &e.bar[s], pcol, prow0 + s * kTile);
+    }
+  }
+  float acc[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) acc[t] = 0.0f;
+  for (int s = 0; s < ks; ++s) {
+    // partial s+2 goes to the buffer of partial s-1, which every lane has summed
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && s + 2 < ks) {
+      const int slot = (s + 2) % kEpiBufs;
+      mbar_arrive_expect_tx(&e.bar[slot], kEpiChunkBytes);
+      tma_load_2d(e.base + slot * kEpiChunkBytes, pmap, &e.bar[slot], pcol, prow0 + (s + 2) * kTile);
+    }
+    const int slot = s % kEpiBufs;
+    const bool ok = mbar_wait(&e.bar[slot], (e.parity >> slot) & 1u, abort_flag, p.status,
+                              p.wait_limit_ns);
+    e.parity ^= 1u << slot;
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    const uint8_t* b = e.base + slot * kEpiChunkBytes;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const float4 v = *reinterpret_cast<const float4*>(b + swz128_off(lane, g));
+      acc[4 * g] += v.x;
+      acc[4 * g + 1] += v.y;
+      acc[4 * g + 2] += v.z;
+      acc[4 * g + 3] += v.w;
+    }
+  }
+  __syncwarp();
+  uint32_t bits[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) bits[t] = __float_as_uint(acc[t]);
+  uint8_t* buf = e.base;  // every load has been consumed
+  const bool mirror = T.n0 != T.m0;
+  const int r0 = T.m0 + kBM * rank + 32 * q;
+  const int c0 = T.n0 + half * 128 + kEpiCols * T.sub;
+  epi_sym(T, bp, buf, lane, mirror, bits);
+  epi_store(p, T, bp, buf, r0, c0, lane, mirror);
+  return true;
 }
 
 // Waits that ignore the abort flag, used only to drain in-flight work.
@@ -357,7 +490,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t rank = cluster_ctarank();  // 0: pair leader, issues the MMAs
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
-  const int ntiles = p.ns_steps * (2 * p.sym_begin[p.nbanks] + p.apply_begin[p.nbanks]);
+  const int ntiles = p.ns_steps * tiles_per_step(p);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -399,6 +532,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       bool first = true;
       for (int tile = pair; ok && tile < ntiles; tile += npairs) {
         const Tile T = decode_tile(p, tile);
+        if (T.phase == kReduce) continue;  // no MMA: the epilogue warps sum partials
         const CUtensorMap* amap = &p.maps[T.bank][T.a_map];
         const CUtensorMap* bmap = &p.maps[T.bank][T.b_map];
         // the operands of this tile are final once the phase it reads is done
@@ -417,9 +551,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             uint8_t* st = tiles + stage * kStageBytes;
             const uint32_t bar = full_leader + 8u * static_cast<uint32_t>(stage);
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
-            load_operand(st, amap, bar, T.a_mn, T.a_base, T.m0 + kBM * rank, kb * kBK);
-            load_operand(st + kATileBytes, bmap, bar, T.b_mn, T.b_base, T.n0 + (kBN / 2) * rank,
-                         kb * kBK);
+            const int k0 = (T.kb0 + kb) * kBK;
+            load_operand(st, amap, bar, T.a_mn, T.a_base, T.m0 + kBM * rank, k0);
+            load_operand(st + kATileBytes, bmap, bar, T.b_mn, T.b_base, T.n0 + (kBN / 2) * rank, k0);
             issued_parity[stage] = static_cast<int>(phase);
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -441,6 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         bool ok = true;
         for (int tile = pair; ok && tile < ntiles; tile += npairs) {
           const Tile T = decode_tile(p, tile);
+          if (T.phase == kReduce) continue;
           const uint32_t idesc = idesc_bf16(2 * kBM, kBN, T.a_mn, T.b_mn);
           if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, limit)) {
             ok = false;
@@ -490,6 +625,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = pair; ok && tile < ntiles; tile += npairs) {
       const Tile T = decode_tile(p, tile);
       const BankPlan& bp = p.bank[T.bank];
+      if (T.phase == kReduce) {  // no accumulator: sum the split partials
+        if (lane == 0 && !wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit))
+          ok = false;
+        if (!__all_sync(0xffffffffu, ok)) break;
+        if (!epi_reduce(p, e, T, bp, lane, static_cast<int>(rank), q, half, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          bulk_wait_all();
+          fence_proxy_async_global();
+          red_release_gpu_add(T.done_cnt, 1);
+        }
+        __syncwarp();
+        continue;
+      }
+      const bool split = T.phase == kGram && bp.ksplit > 1;
+      const int prow = (T.mat * bp.tiles_sym + T.sym_t) * bp.ksplit * kTile + T.split * kTile +
+                       kBM * static_cast<int>(rank) + 32 * q;
       const int r0 = T.m0 + kBM * static_cast<int>(rank) + 32 * q;  // first row of this warp
       const int cw = T.n0 + half * 128;                              // first column of this warp
       const bool mirror = T.phase != kApply && T.n0 != T.m0;
@@ -531,11 +685,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         tmem_ld_wait();
         uint8_t* buf = ring_buf(e, k);
-        if (T.phase == kApply)
-          epi_apply(T, bp, buf, lane, r);
-        else
-          epi_sym(T, bp, buf, lane, mirror, r);
-        epi_store(p, T, bp, buf, r0, c0, lane, mirror);
+        if (split) {
+          epi_partial(p, T, buf, lane, prow, half * 128 + j * kEpiCols, r);
+        } else {
+          if (T.phase == kApply)
+            epi_apply(T, bp, buf, lane, r);
+          else
+            epi_sym(T, bp, buf, lane, mirror, r);
+          epi_store(p, T, bp, buf, r0, c0, lane, mirror);
+        }
         e.chunk = k + 1;
       }
       if (!ok) break;
@@ -572,7 +730,7 @@ cudaError_t ns_gemm_prepare() {
 }
 
 cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s) {
-  const int tiles = p.ns_steps * (2 * p.sym_begin[p.nbanks] + p.apply_begin[p.nbanks]);
+  const int tiles = p.ns_steps * tiles_per_step(p);
   int pairs = num_sms / 2;
   if (tiles < pairs) pairs = tiles;
   if (pairs < 1) pairs = 1;

@@ -36,9 +36,11 @@ constexpr int kEpiBufBytes = kEpiBufs * kEpiChunkBytes;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 1024 + 512;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, then epilogue
 constexpr int kChunk = 8192;       // padded elements per block in the momentum pass
-constexpr int kMaxMaps = 13;
+constexpr int kMaxMaps = 14;
 
-enum Phase : int { kGram = 0, kPoly = 1, kApply = 2 };
+enum Phase : int { kGram = 0, kPoly = 1, kApply = 2, kReduce = 3 };
+constexpr int kRedSub = 4;         // reduce sub-tiles per 256 x 256 tile (32 columns per warp)
+constexpr int kMaxSplit = 16;      // K splits of a Gram product
 
 // Tensor-map slots per bank. Operand maps (128-byte swizzle): K-major boxes
 // of 128 rows x 64 columns, MN-major boxes of 64 x 64. Epilogue maps: 32 x 32
@@ -46,7 +48,8 @@ enum Phase : int { kGram = 0, kPoly = 1, kApply = 2 };
 // mirror chunks of A and B.
 enum MapSlot : int {
   kHiK0 = 0, kHiK1 = 1, kHiMN0 = 2, kHiMN1 = 3, kAK = 4, kBK_ = 5,
-  kHiE0 = 6, kHiE1 = 7, kLoE = 8, kAE = 9, kAT = 10, kBE = 11, kBT = 12
+  kHiE0 = 6, kHiE1 = 7, kLoE = 8, kAE = 9, kAT = 10, kBE = 11, kBT = 12,
+  kPartE = 13  // fp32 Gram partial tiles, 32 x 32 boxes, 128-byte swizzle
 };
 
 struct BankPlan {
@@ -54,26 +57,35 @@ struct BankPlan {
   int chunks;                   // momentum-pass blocks per matrix
   int tiles_sym;                // upper 256x256 tiles of an rp x rp symmetric product
   int tiles_apply;              // (Rp/256) * (Cp/256)
+  int ksplit;                   // K splits of the Gram product (1: none)
+  int kc;                       // 64-deep K blocks per split
+  int tiles_red;                // reduce sub-tiles (tiles_sym * kRedSub when split)
   __nv_bfloat16* hi[2];         // iterate, high bf16 part (ping-pong)
   __nv_bfloat16* lo;            // iterate, low bf16 part (in place)
   __nv_bfloat16* A;             // Gram matrix, count x rp x rp
   __nv_bfloat16* B;             // b A + c A^2, count x rp x rp
   float* partial;               // count x chunks sums of squares
   float* scale;                 // count: 1 / (||U||_F + eps)
-  int* counters;                // count x 3: finished tile parts of Gram, Poly, Apply
+  int* counters;                // count x 4: finished tile parts of Gram, Poly, Apply, Reduce
+  float* part;                  // fp32 Gram partials [count][tiles_sym][ksplit][256][256]
 };
 
 // ---------------------------------------------------------------- GEMM chain
 // One persistent launch runs every Newton-Schulz step of every matrix. Tiles
-// are listed step by step, phase by phase, bank by bank, matrix by matrix;
-// CTA pairs take them round-robin. A tile waits on per-matrix counters for
-// the phase it reads; every epilogue warp of both CTAs adds 1 to its own
-// phase's counter when its stores are complete (kTileParts per tile).
+// are listed step by step, phase by phase (Gram, Reduce, Poly, Apply), bank by
+// bank, matrix by matrix; CTA pairs take them round-robin. A tile waits on
+// per-matrix counters for the phase it reads; every epilogue warp of both
+// CTAs adds 1 to its own phase's counter when its stores are complete
+// (kTileParts per tile). Banks whose Gram K is much longer than the matrix is
+// wide split that product along K: the split tiles store fp32 partials and
+// Reduce sub-tiles sum them into A.
 constexpr int kTileParts = 2 * kEpiWarps;
 
 struct NsGemmParams {
   CUtensorMap maps[MUON_MAX_BANKS][kMaxMaps];
   BankPlan bank[MUON_MAX_BANKS];
+  int gram_begin[MUON_MAX_BANKS + 1];   // prefix sums of count * tiles_sym * ksplit
+  int red_begin[MUON_MAX_BANKS + 1];    // prefix sums of count * tiles_red
   int sym_begin[MUON_MAX_BANKS + 1];    // prefix sums of count * tiles_sym
   int apply_begin[MUON_MAX_BANKS + 1];  // prefix sums of count * tiles_apply
   int nbanks;
