@@ -45,7 +45,7 @@ def _args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
                     help="1..5 (default 2, the GPT-124M bank the metric names); the others "
@@ -332,28 +332,60 @@ def run_native(args):
     post_gbs = elem_bytes * post_b / (statistics.mean(post_ms) * 1e-3) / 1e9
 
     # -------- end to end through the public API with host buffers
+    # Every step uploads its gradients from pinned host memory and reads the
+    # updated parameters back, pipelined the way a training loop would: the
+    # upload of step s+1 (its own device gradient buffer) and the read-back of
+    # step s-1 (from an on-device snapshot of the parameters) run on two copy
+    # streams while step s computes.
     e2e = None
     if rank == 0 or world > 1:
-        host_params = [torch.empty(bk.param.shape, dtype=bk.param.dtype).pin_memory() for bk in banks]
-        h2d = sum(g.numel() * g.element_size() for g in host_grads)
-        d2h = sum(p.numel() * p.element_size() for p in host_params)
         E = args.e2e_steps
+        up_s, down_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        gbufs = [[torch.empty_like(bk.grad) for bk in banks] for _ in range(2)]
+        snaps = [[torch.empty_like(bk.param) for bk in banks] for _ in range(2)]
+        host_params = [[torch.empty(bk.param.shape, dtype=bk.param.dtype).pin_memory()
+                        for bk in banks] for _ in range(2)]
+        bank_sets = [[mb.Bank(bk.param, g, bk.momentum, bk.momentum_slow, bk.ema)
+                      for bk, g in zip(banks, gb)] for gb in gbufs]
+        h2d = sum(g.numel() * g.element_size() for g in host_grads)
+        d2h = sum(p_.numel() * p_.element_size() for p_ in host_params[0])
+        up_done = [torch.cuda.Event() for _ in range(2)]
+        grads_free = [torch.cuda.Event() for _ in range(2)]
+        snap_done = [torch.cuda.Event() for _ in range(2)]
+        down_done = [torch.cuda.Event() for _ in range(2)]
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for s in range(E):
-            for bk, g in zip(banks, host_grads):
-                bk.grad.copy_(g, non_blocking=True)
-            step_fn(banks, H, ws)
-            for bk, hp_ in zip(banks, host_params):
-                hp_.copy_(bk.param, non_blocking=True)
+        for s_ in range(E):
+            i = s_ % 2
+            up_s.wait_event(e0 if s_ < 2 else grads_free[i])  # step s-2 has consumed buffer i
+            with torch.cuda.stream(up_s):
+                for gb, g in zip(gbufs[i], host_grads):
+                    gb.copy_(g, non_blocking=True)
+            up_done[i].record(up_s)
+            stream.wait_event(up_done[i])
+            step_fn(bank_sets[i], H, ws)
+            grads_free[i].record(stream)
+            if s_ >= 2:
+                stream.wait_event(down_done[i])  # snapshot i has been read back
+            for sn, bk in zip(snaps[i], banks):
+                sn.copy_(bk.param, non_blocking=True)
+            snap_done[i].record(stream)
+            down_s.wait_event(snap_done[i])
+            with torch.cuda.stream(down_s):
+                for hp_, sn in zip(host_params[i], snaps[i]):
+                    hp_.copy_(sn, non_blocking=True)
+            down_done[i].record(down_s)
+        for i in range(min(E, 2)):
+            stream.wait_event(down_done[(E - 1 - i) % 2])
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
         e2e = {"value": job_throughput(world, E, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
-               "what": "per step: pinned host->device copy of the bf16 gradients, muon_step, "
-                       "device->host copy of the updated bf16 parameters"}
+               "what": "per step: pinned host->device copy of the gradients, the optimizer step "
+                       "through the public API, device->host copy of the updated parameters; "
+                       "copies of neighbouring steps overlap the step on two copy streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

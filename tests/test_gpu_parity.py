@@ -172,16 +172,21 @@ def test_anvil_steps_ema_and_readout_blend():
         banks.append(mb.Bank(th, None, z.clone(), z.clone(), th.float().clone()))
     ws = mb.alloc_workspace([bk.shape for bk in banks])
     H = mb.Hparams.from_dict(hp)
-    steps = 3
+    steps = w.steps  # 50: the averaging window of the workload
+    checked = {0, 1, steps // 2, steps - 1}
     for step in range(steps):
         grads = [mi.make_grads(w, b, step) for b in range(len(w.banks))]
-        old = [(bk.param.clone(), bk.momentum.clone(), bk.momentum_slow.clone(), bk.ema.clone())
-               for bk in banks]
+        check = step in checked
+        if check:
+            old = [(bk.param.clone(), bk.momentum.clone(), bk.momentum_slow.clone(), bk.ema.clone())
+                   for bk in banks]
         for bk, g in zip(banks, grads):
             bk.grad = g.to(DEV)
         mb.anvil_step(banks, H, ws)
         torch.cuda.synchronize()
         assert mb.device_status(ws) == 0
+        if not check:
+            continue
         for b, bk in enumerate(banks):
             th0, Mf0, Ms0, E0 = old[b]
             G = f64(grads[b])
@@ -205,6 +210,10 @@ def test_anvil_steps_ema_and_readout_blend():
                                               oracle.shape_scale(R, C)) - t0
                 ok, r = delta_ok(t0, f64(bk.param[i]), dref, "bf16")
                 assert ok, ("anvil delta", b, i, r)
+                # six polynomial applications on the GPU's own fast momentum
+                Og = f64(orth_gpu(bk.momentum[i:i + 1].clone(), hp["coeffs"])[0])
+                assert rel_fro(Og, O) <= TOL_UPDATE, ("anvil O", b, i, rel_fro(Og, O))
+                assert sv_maxdiff(Og, O) <= TOL_SV
     # readout blend on the 768 x 50304 readout
     rd = banks[-1]
     out = torch.empty_like(rd.param)
