@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define MUON_ABI_VERSION 1
+#define MUON_ABI_VERSION 2
 #define MUON_MAX_NS_STEPS 16
 #define MUON_MAX_BANKS 8
 
@@ -90,6 +90,11 @@ typedef struct {
   float ema_beta;           /* 0 <= beta < 1; used when a bank has ema != NULL        */
   float beta_fast;          /* ANVIL fast-momentum beta, 0 <= beta < 1                */
   float beta_slow;          /* ANVIL slow-momentum beta, 0 <= beta < 1                */
+  int32_t sgd_momentum;     /* Muon only. 0: moving average M <- mu M + (1-mu) G
+                             * (Nesterov U = (1-mu) G + mu M); 1: SGD form
+                             * M <- mu M + G (Nesterov U = G + mu M). From zero state
+                             * the SGD buffer is the moving average / (1 - mu), so
+                             * both forms give the same update O.               */
 } muon_hparams;
 
 /* ABI version of the loaded library (MUON_ABI_VERSION). */

@@ -58,7 +58,8 @@ class CHparams(ctypes.Structure):
                 ("weight_decay", ctypes.c_float), ("eps", ctypes.c_float),
                 ("nesterov", ctypes.c_int32), ("ns_steps", ctypes.c_int32),
                 ("coeffs", ctypes.c_float * (3 * MAX_NS_STEPS)), ("ema_beta", ctypes.c_float),
-                ("beta_fast", ctypes.c_float), ("beta_slow", ctypes.c_float)]
+                ("beta_fast", ctypes.c_float), ("beta_slow", ctypes.c_float),
+                ("sgd_momentum", ctypes.c_int32)]
 
 
 _vp, _i32, _i64, _sz, _f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -127,11 +128,12 @@ class Hparams:
     ema_beta: float = 0.99
     beta_fast: float = 0.9
     beta_slow: float = 0.99
+    sgd_momentum: bool = False
 
     @classmethod
     def from_dict(cls, d: dict) -> "Hparams":
         keys = {k: d[k] for k in ("lr", "mu", "weight_decay", "eps", "nesterov", "coeffs",
-                                  "ema_beta", "beta_fast", "beta_slow") if k in d}
+                                  "ema_beta", "beta_fast", "beta_slow", "sgd_momentum") if k in d}
         return cls(**keys)
 
     def to_c(self) -> CHparams:
@@ -144,6 +146,7 @@ class Hparams:
         for i, (a, b, c) in enumerate(list(self.coeffs)[:MAX_NS_STEPS]):
             h.coeffs[3 * i], h.coeffs[3 * i + 1], h.coeffs[3 * i + 2] = a, b, c
         h.ema_beta, h.beta_fast, h.beta_slow = self.ema_beta, self.beta_fast, self.beta_slow
+        h.sgd_momentum = 1 if self.sgd_momentum else 0
         return h
 
 

@@ -268,6 +268,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   mp.mu = v == Variant::kAnvil ? hp->beta_fast : hp->mu;
   mp.mu_slow = hp->beta_slow;
   mp.nesterov = hp->nesterov ? 1 : 0;
+  mp.sgd = (v == Variant::kMuon && hp->sgd_momentum) ? 1 : 0;
   mp.eps = hp->eps;
   int blocks = 0, mats = 0;
   for (int b = 0; b < nbanks; ++b) {

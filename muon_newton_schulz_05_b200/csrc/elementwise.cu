@@ -75,8 +75,9 @@ __device__ __forceinline__ float momentum_elem(const MomParams& p, float g, floa
     ms = fmaf(p.mu_slow, ms, (1.0f - p.mu_slow) * g);
     return m;
   }
-  m = fmaf(p.mu, m, (1.0f - p.mu) * g);
-  return p.nesterov ? fmaf(p.mu, m, (1.0f - p.mu) * g) : m;
+  const float gw = p.sgd ? g : (1.0f - p.mu) * g;  // SGD form or moving average
+  m = fmaf(p.mu, m, gw);
+  return p.nesterov ? fmaf(p.mu, m, gw) : m;
 }
 
 __device__ __forceinline__ float block_sum_256(float v, float* red) {
@@ -215,29 +216,83 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
     const __nv_bfloat16* hi = bp.hi[p.final_buf];
     const __nv_bfloat16* lo = bp.lo;
     const long long padded = static_cast<long long>(bp.Rp) * bp.Cp;
-    if ((bp.C & 7) == 0) {
-      for (long long g = tid; g < n / 8; g += nthr) {
+    const unsigned long long ngroups = static_cast<unsigned long long>(n / 8);
+    if ((bp.C & 7) == 0 && ngroups < (1ull << 32)) {
+      // groups of 8 consecutive elements of a row; 32-bit index arithmetic and
+      // two independent groups per thread per pass (all loads issued first)
+      const uint32_t ng = static_cast<uint32_t>(ngroups);
+      const uint32_t gpr = static_cast<uint32_t>(bp.C / 8);
+      const uint32_t R = static_cast<uint32_t>(bp.R);
+      const uint32_t t32 = static_cast<uint32_t>(tid), n32 = static_cast<uint32_t>(nthr);
+      for (uint32_t g0 = t32; g0 < ng; g0 += 2 * n32) {
+        long long e[2], off[2];
+        bool has[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const uint32_t g = g0 + static_cast<uint32_t>(u) * n32;
+          has[u] = g < ng;
+          const uint32_t gg = has[u] ? g : g0;
+          const uint32_t row = gg / gpr;
+          const uint32_t col = (gg - row * gpr) * 8u;
+          const uint32_t mat = row / R;
+          const uint32_t r = row - mat * R;
+          e[u] = static_cast<long long>(gg) * 8;
+          off[u] = (static_cast<long long>(mat) * bp.Rp + r) * bp.Cp + col;
+        }
+        float o[2][8], th[2][8], ms[2][8];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (!has[u]) continue;
+          load8(hi, MUON_BF16, off[u], o[u]);
+          if (p.mode != kUpdWriteO) load8(io.param, io.param_dtype, e[u], th[u]);
+          if (p.mode == kUpdCautious) load8(io.mom_slow, MUON_F32, e[u], ms[u]);
+          if (p.use_lo) {
+            float l8[8];
+            load8(lo, MUON_BF16, off[u], l8);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) o[u][t] += l8[t];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (!has[u]) continue;
+          if (p.mode == kUpdWriteO) {
+            store8(io.param, io.param_dtype, e[u], o[u]);
+            continue;
+          }
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            th[u][t] = stored(io.param_dtype,
+                              update_elem(p, io, th[u][t], o[u][t], p.mode == kUpdCautious ? ms[u][t] : 0.0f));
+          store8(io.param, io.param_dtype, e[u], th[u]);
+          if (io.ema) {
+            float em[8];
+            load8(io.ema, MUON_F32, e[u], em);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) em[t] = fmaf(p.ema_beta, em[t], (1.0f - p.ema_beta) * th[u][t]);
+            store8(io.ema, MUON_F32, e[u], em);
+          }
+        }
+      }
+    } else if ((bp.C & 7) == 0) {
+      for (long long g = tid; g < n / 8; g += nthr) {  // banks beyond 2^35 elements
         const long long e = g * 8;
         const long long mat = e / per;
         const long long rem = e - mat * per;
         const long long row = rem / bp.C;
-        const long long col = rem - row * bp.C;
-        const long long off = mat * padded + row * bp.Cp + col;
-        float o[8], h8[8], l8[8];
-        load8(hi, MUON_BF16, off, h8);
+        const long long off = mat * padded + row * bp.Cp + (rem - row * bp.C);
+        float o[8], th[8], ms[8];
+        load8(hi, MUON_BF16, off, o);
         if (p.use_lo) {
+          float l8[8];
           load8(lo, MUON_BF16, off, l8);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) o[t] = h8[t] + l8[t];
-        } else {
-#pragma unroll
-          for (int t = 0; t < 8; ++t) o[t] = h8[t];
+          for (int t = 0; t < 8; ++t) o[t] += l8[t];
         }
         if (p.mode == kUpdWriteO) {
           store8(io.param, io.param_dtype, e, o);
           continue;
         }
-        float th[8], ms[8];
         load8(io.param, io.param_dtype, e, th);
         if (p.mode == kUpdCautious) load8(io.mom_slow, MUON_F32, e, ms);
 #pragma unroll
@@ -274,8 +329,8 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
 }
 
 cudaError_t launch_update(const UpdParams& p, long long total_elems, int num_sms, cudaStream_t s) {
-  long long want = (total_elems / 8 + 255) / 256;
-  int grid = static_cast<int>(want < 1 ? 1 : (want > 16LL * num_sms ? 16LL * num_sms : want));
+  long long want = (total_elems / 16 + 255) / 256;  // two groups of 8 per thread per pass
+  int grid = static_cast<int>(want < 1 ? 1 : (want > 8LL * num_sms ? 8LL * num_sms : want));
   update_kernel<<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }

@@ -116,6 +116,7 @@ struct MomParams {
   float mu;           // Muon mu, or ANVIL beta_fast
   float mu_slow;      // ANVIL beta_slow
   int nesterov;
+  int sgd;            // Muon SGD-form momentum (M <- mu M + G)
   float eps;
   int mat_begin[MUON_MAX_BANKS + 1];
 };

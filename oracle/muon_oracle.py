@@ -60,7 +60,9 @@ __all__ = [
     "round_to_bf16",
     "round_to_storage",
     "momentum_update",
+    "momentum_update_sgd",
     "nesterov_lookahead",
+    "nesterov_lookahead_sgd",
     "frobenius_normalize",
     "newton_schulz",
     "orthogonalize",
@@ -122,6 +124,20 @@ def momentum_update(M: np.ndarray, G: np.ndarray, mu: float) -> np.ndarray:
     [P1] "Muonとは" calls the momentum a moving average of the gradient (R1).
     """
     return mu * M + (1.0 - mu) * G
+
+
+def momentum_update_sgd(M: np.ndarray, G: np.ndarray, mu: float) -> np.ndarray:
+    """SGD-form momentum M <- mu M + G (the "SGD-momentum" of "Muonが登場"),
+    the alternative to R1 that a flag selects."""
+    return mu * M + G
+
+
+def nesterov_lookahead_sgd(M_new: np.ndarray, G: np.ndarray, mu: float,
+                           nesterov: bool) -> np.ndarray:
+    """U = G + mu M for the SGD form with Nesterov, else U = M."""
+    if nesterov:
+        return G + mu * M_new
+    return M_new
 
 
 def nesterov_lookahead(M_new: np.ndarray, G: np.ndarray, mu: float,
@@ -196,15 +212,20 @@ def cautious_update(theta: np.ndarray, O: np.ndarray, mask: np.ndarray,
 def muon_step(theta, G, M, hp: dict, param_dtype: str):
     """One Muon step on one matrix.
 
-    hp keys: lr, mu, weight_decay, nesterov, coeffs (list of (a, b, c)), eps.
+    hp keys: lr, mu, weight_decay, nesterov, coeffs (list of (a, b, c)), eps,
+    and optionally sgd_momentum (SGD-form buffer instead of the moving average).
     Returns (theta_new rounded to param_dtype, M_new, O).
     """
     theta = as_f64(theta)
     G = as_f64(G)
     M = as_f64(M)
     rows, cols = theta.shape
-    M_new = momentum_update(M, G, hp["mu"])
-    U = nesterov_lookahead(M_new, G, hp["mu"], bool(hp["nesterov"]))
+    if hp.get("sgd_momentum"):
+        M_new = momentum_update_sgd(M, G, hp["mu"])
+        U = nesterov_lookahead_sgd(M_new, G, hp["mu"], bool(hp["nesterov"]))
+    else:
+        M_new = momentum_update(M, G, hp["mu"])
+        U = nesterov_lookahead(M_new, G, hp["mu"], bool(hp["nesterov"]))
     O = orthogonalize(U, hp["coeffs"], hp["eps"])
     theta_new = decoupled_update(theta, O, hp["lr"], hp["weight_decay"],
                                  shape_scale(rows, cols))

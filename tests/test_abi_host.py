@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strings():
-    assert mb.abi_version() == 1
+    assert mb.abi_version() == 2
     for code, name in mb.STATUS_NAMES.items():
         assert mb.status_string(code).startswith(name)
     assert "unknown" in mb.status_string(77)
@@ -48,9 +48,9 @@ def test_struct_layout_matches_header():
 #include <stddef.h>
 #include "muon_b200.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(muon_bank), offsetof(muon_bank, grad),
+  printf("%zu %zu %zu %zu %zu %zu %zu\n", sizeof(muon_bank), offsetof(muon_bank, grad),
          offsetof(muon_bank, ema), sizeof(muon_hparams), offsetof(muon_hparams, coeffs),
-         offsetof(muon_hparams, beta_slow));
+         offsetof(muon_hparams, beta_slow), offsetof(muon_hparams, sgd_momentum));
   return 0;
 }
 '''
@@ -61,7 +61,8 @@ int main(void) {
         subprocess.check_call(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), c, "-o", exe])
         got = [int(x) for x in subprocess.check_output([exe]).split()]
     want = [ctypes.sizeof(mb.CBank), mb.CBank.grad.offset, mb.CBank.ema.offset,
-            ctypes.sizeof(mb.CHparams), mb.CHparams.coeffs.offset, mb.CHparams.beta_slow.offset]
+            ctypes.sizeof(mb.CHparams), mb.CHparams.coeffs.offset, mb.CHparams.beta_slow.offset,
+            mb.CHparams.sgd_momentum.offset]
     assert got == want
 
 

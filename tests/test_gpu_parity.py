@@ -116,14 +116,17 @@ def _muon_run(w, steps, check_steps, sample, hp_override=None):
             th0, M0 = old[b]
             G = grads[b]
             # momentum on every element
-            Mref = oracle.momentum_update(f64(M0), f64(G), hp["mu"])
+            sgd = bool(hp.get("sgd_momentum"))
+            upd = oracle.momentum_update_sgd if sgd else oracle.momentum_update
+            look = oracle.nesterov_lookahead_sgd if sgd else oracle.nesterov_lookahead
+            Mref = upd(f64(M0), f64(G), hp["mu"])
             ok, r = buffer_ok(f64(bk.momentum), Mref, TOL_BUFFER)
             assert ok, ("momentum", b, step, r)
             R, C = bk.shape[1:]
             s = oracle.shape_scale(R, C)
             tol_o, tol_sv = update_tols(R, C)
             for i in sample(b, bk.shape[0]):
-                U = oracle.nesterov_lookahead(Mref[i], f64(G[i]), hp["mu"], bool(hp["nesterov"]))
+                U = look(Mref[i], f64(G[i]), hp["mu"], bool(hp["nesterov"]))
                 O = oracle.orthogonalize(U, hp["coeffs"], hp["eps"])
                 # the NS path on the GPU's own U
                 Ug = torch.from_numpy(U.astype(np.float32))[None].to(DEV)
@@ -151,6 +154,13 @@ def test_gpt124m_bank_ten_steps():
 def test_square_1024_bank_with_decay():
     w = mi.workloads()[3]
     _muon_run(w, 3, {0, 2}, lambda b, n: [0, 37])
+
+
+def test_sgd_form_momentum_flag():
+    w = mi.custom_workload([(4, 512, 768), (2, 768, 512)],
+                           dict(lr=0.02, mu=0.9, weight_decay=0.05, nesterov=1,
+                                coeffs=[QUINTIC] * 5, eps=1e-7, sgd_momentum=1), cid=93)
+    _muon_run(w, 3, {0, 2}, lambda b, n: [0, n - 1])
 
 
 def test_ragged_bank_mix():

@@ -134,6 +134,28 @@ def test_momentum_three_step_unroll():
     assert oracle.nesterov_lookahead(M, G3, mu, False) is M
 
 
+def test_sgd_form_three_step_unroll_and_step():
+    rng = np.random.default_rng(31)
+    G1, G2, G3 = (rng.standard_normal((2, 3)) for _ in range(3))
+    mu = 0.9
+    M = np.zeros((2, 3))
+    for G in (G1, G2, G3):
+        M = oracle.momentum_update_sgd(M, G, mu)
+    assert np.max(np.abs(M - (G3 + mu * G2 + mu * mu * G1))) < 1e-15
+    U = oracle.nesterov_lookahead_sgd(M, G3, mu, True)
+    assert np.max(np.abs(U - (G3 + mu * (G3 + mu * G2 + mu * mu * G1)))) < 1e-15
+    # through muon_step: the SGD buffer is (1 - mu)^-1 times the moving average
+    # and the orthogonalised update is the same
+    th = rng.standard_normal((6, 10))
+    G = rng.standard_normal((6, 10))
+    hp = dict(lr=0.02, mu=mu, weight_decay=0.0, nesterov=1, coeffs=[QUINTIC] * 5, eps=0.0)
+    t_ma, M_ma, O_ma = oracle.muon_step(th, G, np.zeros((6, 10)), hp, "f32")
+    t_sg, M_sg, O_sg = oracle.muon_step(th, G, np.zeros((6, 10)), dict(hp, sgd_momentum=1), "f32")
+    assert np.allclose(M_sg * (1 - mu), M_ma, atol=1e-14)
+    assert np.max(np.abs(O_sg - O_ma)) < 1e-12
+    assert np.array_equal(t_sg, t_ma)
+
+
 def test_sgd_momentum_form_gives_the_same_update():
     """From zero state the SGD form M' = mu M' + G is M / (1 - mu); the
     normalisation removes the factor, so O is the same (reading R1)."""
