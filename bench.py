@@ -36,7 +36,7 @@ LAUNCHES_PER_STEP = 4
 # DRAM bytes (read + write) of one Newton-Schulz chain launch on this workload,
 # from the ncu capture summarised in profiles/ns_gemm_gpt124m_bank.md. Set to
 # None whenever ns_gemm_kernel changes until it is captured again.
-NS_CHAIN_DRAM_BYTES = 5.815693e9
+NS_CHAIN_DRAM_BYTES = 5.889017e9
 
 
 def _args():

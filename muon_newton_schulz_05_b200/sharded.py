@@ -1,0 +1,256 @@
+"""Data-parallel Muon over a process group: each matrix has one owner rank.
+
+In data-parallel training every rank holds the whole bank and its own
+gradient. Muon's matrix products can be spread over the GPUs layer by layer
+(page "きみはNanoGPT speedrunを知っているか？", section "おまけ"). Here every
+matrix gets one owner, chosen so that the ranks' Newton-Schulz flops
+(3 r^2 c + r^3 per iteration, r <= c the short side) come out balanced:
+largest first, each to the least-loaded rank. One step, per bucket of banks:
+
+  1. reduce-scatter: gradients packed in owner order are averaged over the
+     ranks; each rank receives the gradients of the matrices it owns;
+  2. the owner runs the optimizer step (the CUDA library) on its matrices
+     only, so momentum and workspace live on one rank;
+  3. all-gather: the owners' updated parameters reach every rank, which
+     unpacks them into its bank.
+
+All reduce-scatters are issued at once (asynchronous); bucket k's step waits
+only for bucket k's, so on NCCL the exchange of later buckets overlaps the
+Newton-Schulz chain of earlier ones, and each bucket's all-gather overlaps
+the next bucket's step. The packing and unpacking are plain copies; every
+arithmetic step of the optimizer runs in the library's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Callable, List, Optional, Sequence, Tuple
+
+# every bank's slot in a segment starts on a 256-byte boundary (the library
+# wants 16-byte aligned operands; 256 also keeps NCCL on its vector path)
+_ALIGN_ELEMS = 128
+
+
+def ns_work(rows: int, cols: int) -> float:
+    """Newton-Schulz flops of one iteration on a rows x cols matrix, over 2."""
+    r, c = min(rows, cols), max(rows, cols)
+    return 3.0 * r * r * c + float(r) ** 3
+
+
+def _round_up(x: int, m: int) -> int:
+    return (x + m - 1) // m * m
+
+
+@dataclass
+class Bucket:
+    banks: List[int]                 # bank indices in this bucket
+    owned: List[List[List[int]]]     # owned[rank][j] = matrix indices of banks[j]
+    offsets: List[List[int]]         # offsets[rank][j] = element offset in the segment
+    seg: int                         # elements per rank segment (padded)
+
+
+@dataclass
+class ShardPlan:
+    world: int
+    shapes: List[Tuple[int, int, int]]
+    owner: List[List[int]]           # owner[b][i]
+    buckets: List[Bucket]
+    load: List[float]                # per-rank Newton-Schulz work
+
+    @classmethod
+    def build(cls, shapes: Sequence[Tuple[int, int, int]], world: int,
+              buckets: Optional[Sequence[Sequence[int]]] = None) -> "ShardPlan":
+        """buckets: lists of bank indices (default: one bucket with all banks).
+        Owners are assigned bucket by bucket with the load carried over, so
+        each bucket and the whole step are both close to balanced."""
+        shapes = [tuple(int(v) for v in s) for s in shapes]
+        if world < 1:
+            raise ValueError("world size must be >= 1")
+        groups = [list(g) for g in buckets] if buckets is not None else [list(range(len(shapes)))]
+        seen = sorted(b for g in groups for b in g)
+        if seen != list(range(len(shapes))):
+            raise ValueError("buckets must list every bank exactly once")
+        load = [0.0] * world
+        owner = [[0] * s[0] for s in shapes]
+        out = []
+        for g in groups:
+            items = sorted(((-ns_work(shapes[b][1], shapes[b][2]), b, i)
+                            for b in g for i in range(shapes[b][0])))
+            for negw, b, i in items:
+                r = min(range(world), key=lambda k: (load[k], k))
+                owner[b][i] = r
+                load[r] -= negw
+            owned = [[[i for i in range(shapes[b][0]) if owner[b][i] == r] for b in g]
+                     for r in range(world)]
+            offsets, seg = [], 0
+            for r in range(world):
+                pos, offs = 0, []
+                for j, b in enumerate(g):
+                    offs.append(pos)
+                    pos += _round_up(len(owned[r][j]) * shapes[b][1] * shapes[b][2], _ALIGN_ELEMS)
+                offsets.append(offs)
+                seg = max(seg, pos)
+            out.append(Bucket(g, owned, offsets, max(seg, _ALIGN_ELEMS)))
+        return cls(world, list(shapes), owner, out, load)
+
+    def views(self, k: int, rank: int, seg_flat) -> List:
+        """[n_owned, R, C] views of rank's segment of bucket k, one per bank of
+        the bucket (None where the rank owns no matrix of that bank)."""
+        bk = self.buckets[k]
+        out = []
+        for j, b in enumerate(bk.banks):
+            n = len(bk.owned[rank][j])
+            _, rows, cols = self.shapes[b]
+            o = bk.offsets[rank][j]
+            out.append(seg_flat[o:o + n * rows * cols].view(n, rows, cols) if n else None)
+        return out
+
+    def pack(self, k: int, tensors: Sequence, flat) -> None:
+        """Bank tensors -> flat (world * seg of bucket k), segment r holding
+        rank r's matrices. Padding is left as it is."""
+        seg = self.buckets[k].seg
+        for r in range(self.world):
+            for j, v in enumerate(self.views(k, r, flat[r * seg:(r + 1) * seg])):
+                if v is not None:
+                    v.copy_(tensors[self.buckets[k].banks[j]][self.buckets[k].owned[r][j]])
+
+    def unpack(self, k: int, flat, tensors: Sequence) -> None:
+        """Inverse of pack for bucket k."""
+        seg = self.buckets[k].seg
+        for r in range(self.world):
+            for j, v in enumerate(self.views(k, r, flat[r * seg:(r + 1) * seg])):
+                if v is not None:
+                    tensors[self.buckets[k].banks[j]][self.buckets[k].owned[r][j]] = v
+
+
+class ShardedMuon:
+    """Owner-sharded data-parallel Muon (or ANVIL) step for a list of banks.
+
+    params: this rank's full bank tensors [count, R, C], identical on every
+    rank and overwritten with the updated bank; grads: this rank's local
+    gradients of the same shapes. Each rank keeps fp32 momentum (ANVIL: both
+    momenta, and the EMA when ema=True) for the matrices it owns only.
+    step_fn(banks, hp, workspace) runs the local step on Bank objects and
+    defaults to the library's muon_step (anvil_step for variant="anvil");
+    workspace_fn(shapes) allocates its workspace.
+    """
+
+    def __init__(self, shapes, param_dtype, grad_dtype, group=None, variant: str = "muon",
+                 device=None, buckets=None, ema: bool = False,
+                 step_fn: Optional[Callable] = None, workspace_fn: Optional[Callable] = None):
+        import torch
+        import torch.distributed as dist
+        if variant not in ("muon", "anvil"):
+            raise ValueError("variant must be 'muon' or 'anvil'")
+        self.dist, self.group = dist, group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.gloo = dist.get_backend(group) == "gloo"
+        self.plan = ShardPlan.build(shapes, self.world, buckets)
+        self.variant = variant
+        self.device = device if device is not None else torch.device("cpu")
+        if step_fn is None or workspace_fn is None:
+            from . import alloc_workspace, anvil_step, muon_step
+            step_fn = step_fn or (anvil_step if variant == "anvil" else muon_step)
+            workspace_fn = workspace_fn or (lambda shapes: alloc_workspace(shapes, self.device))
+        self.step_fn, self.workspace_fn = step_fn, workspace_fn
+        self.workspaces: List = [None] * len(self.plan.buckets)
+        self._gflat, self._gseg, self._pflat, self._pseg = [], [], [], []
+        self.momentum, self.momentum_slow, self.ema = [], [], []
+        for k, bk in enumerate(self.plan.buckets):
+            n = self.world * bk.seg
+            self._gflat.append(torch.zeros(n, dtype=grad_dtype, device=self.device))
+            self._gseg.append(torch.zeros(bk.seg, dtype=grad_dtype, device=self.device))
+            self._pflat.append(torch.zeros(n, dtype=param_dtype, device=self.device))
+            self._pseg.append(torch.zeros(bk.seg, dtype=param_dtype, device=self.device))
+
+            def state(on):
+                return [torch.zeros(len(o), *self.plan.shapes[b][1:], dtype=torch.float32,
+                                    device=self.device) if (o and on) else None
+                        for o, b in zip(bk.owned[self.rank], bk.banks)]
+            self.momentum.append(state(True))
+            self.momentum_slow.append(state(variant == "anvil"))
+            self.ema.append(state(ema))
+        self._ema_ready = False
+
+    def owned_shapes(self, k: int) -> List[Tuple[int, int, int]]:
+        bk = self.plan.buckets[k]
+        return [(len(o), *self.plan.shapes[b][1:]) for o, b in zip(bk.owned[self.rank], bk.banks) if o]
+
+    def _reduce_scatter(self, k: int):
+        if self.gloo:
+            # gloo has no reduce-scatter: sum everywhere, keep this rank's segment
+            self.dist.all_reduce(self._gflat[k], op=self.dist.ReduceOp.SUM, group=self.group)
+            seg = self.plan.buckets[k].seg
+            self._gseg[k].copy_(self._gflat[k][self.rank * seg:(self.rank + 1) * seg])
+            self._gseg[k].div_(self.world)
+            return None
+        return self.dist.reduce_scatter_tensor(self._gseg[k], self._gflat[k],
+                                               op=self.dist.ReduceOp.AVG, group=self.group,
+                                               async_op=True)
+
+    def _all_gather(self, k: int):
+        if self.gloo:
+            self.dist.all_gather(list(self._pflat[k].chunk(self.world)), self._pseg[k],
+                                 group=self.group)
+            return None
+        return self.dist.all_gather_into_tensor(self._pflat[k], self._pseg[k],
+                                                group=self.group, async_op=True)
+
+    def step(self, params: Sequence, grads: Sequence, hp) -> None:
+        from . import Bank
+        plan, rank = self.plan, self.rank
+        nb = len(plan.buckets)
+        rs = []
+        for k in range(nb):
+            plan.pack(k, grads, self._gflat[k])
+            rs.append(self._reduce_scatter(k))
+        ag = []
+        for k, bk in enumerate(plan.buckets):
+            if rs[k] is not None:
+                rs[k].wait()
+            gv = plan.views(k, rank, self._gseg[k])
+            pv = plan.views(k, rank, self._pseg[k])
+            banks = []
+            for j, b in enumerate(bk.banks):
+                if pv[j] is None:
+                    continue
+                pv[j].copy_(params[b][bk.owned[rank][j]])
+                banks.append(Bank(pv[j], gv[j], self.momentum[k][j], self.momentum_slow[k][j],
+                                  self.ema[k][j]))
+            if banks:
+                if self.workspaces[k] is None:
+                    self.workspaces[k] = self.workspace_fn([bank.shape for bank in banks])
+                if any(e is not None for e in self.ema[k]):
+                    self._init_ema(k, pv)
+                self.step_fn(banks, hp, self.workspaces[k])
+            ag.append(self._all_gather(k))
+        for k in range(nb):
+            if ag[k] is not None:
+                ag[k].wait()
+            plan.unpack(k, self._pflat[k], params)
+        self._ema_ready = True
+
+    def _init_ema(self, k: int, pv) -> None:
+        # the average starts at the parameters it averages
+        if self._ema_ready:
+            return
+        for e, p in zip(self.ema[k], pv):
+            if e is not None:
+                e.copy_(p)
+
+    def gather_ema(self, out: Sequence) -> None:
+        """Collect the owners' EMA of every matrix into out (fp32 bank tensors)."""
+        import torch
+        for k, bk in enumerate(self.plan.buckets):
+            seg = torch.zeros(bk.seg, dtype=torch.float32, device=self.device)
+            for v, e in zip(self.plan.views(k, self.rank, seg), self.ema[k]):
+                if v is not None:
+                    if e is None:
+                        raise RuntimeError("ShardedMuon was built without ema=True")
+                    v.copy_(e)
+            flat = torch.zeros(self.world * bk.seg, dtype=torch.float32, device=self.device)
+            if self.gloo:
+                self.dist.all_gather(list(flat.chunk(self.world)), seg, group=self.group)
+            else:
+                self.dist.all_gather_into_tensor(flat, seg, group=self.group)
+            self.plan.unpack(k, flat, out)

@@ -1,0 +1,190 @@
+"""Owner-sharded data-parallel Muon on CPU: gloo ranks, the oracle as the local step.
+
+The collective logic (ownership, packing, averaging reduce-scatter, owner
+step, all-gather, unpack) must give every rank the bank that one process
+gets by stepping every matrix on the mean gradient. The local step here is
+the oracle, so the comparison is exact; the library's own step is covered by
+the GPU parity tests.
+"""
+import dataclasses
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+from muon_newton_schulz_05_b200.sharded import ShardPlan, ns_work  # noqa: E402
+
+SHAPES = [(3, 16, 24), (2, 40, 8), (1, 8, 8)]
+GPT_SHAPES = [(48, 768, 768), (12, 768, 3072), (12, 3072, 768)]
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _hp_dict(hp):
+    d = dataclasses.asdict(hp)
+    d["coeffs"] = [tuple(c) for c in d["coeffs"]]
+    return d
+
+
+def _oracle_step_fn(variant):
+    """A local step with the library's signature, computed by the oracle."""
+    from oracle import muon_oracle as oracle
+
+    def step(banks, hp, workspace):
+        h = _hp_dict(hp)
+        for bk in banks:
+            dt = "bf16" if bk.param.dtype == torch.bfloat16 else "f32"
+            for i in range(bk.param.shape[0]):
+                th = bk.param[i].double().numpy()
+                g = bk.grad[i].double().numpy()
+                if variant == "anvil":
+                    t1, mf, ms, _, _ = oracle.anvil_step(th, g, bk.momentum[i].double().numpy(),
+                                                         bk.momentum_slow[i].double().numpy(), h, dt)
+                    bk.momentum_slow[i] = torch.from_numpy(ms).float()
+                    bk.momentum[i] = torch.from_numpy(mf).float()
+                else:
+                    t1, m1, _ = oracle.muon_step(th, g, bk.momentum[i].double().numpy(), h, dt)
+                    bk.momentum[i] = torch.from_numpy(m1).float()
+                bk.param[i] = torch.from_numpy(t1).to(bk.param.dtype)
+                if bk.ema is not None:
+                    e = oracle.ema_update(bk.ema[i].double().numpy(), bk.param[i].double().numpy(),
+                                          hp.ema_beta)
+                    bk.ema[i] = torch.from_numpy(e).float()
+    return step
+
+
+def _hparams(variant):
+    from muon_newton_schulz_05_b200 import Hparams
+    if variant == "anvil":
+        return Hparams(lr=0.05, weight_decay=0.1, coeffs=[(3.4445, -4.7750, 2.0315)] * 6,
+                       beta_fast=0.9, beta_slow=0.99, ema_beta=0.9)
+    return Hparams(lr=0.05, mu=0.95, weight_decay=0.01, nesterov=True)
+
+
+def _params(shapes):
+    g = torch.Generator().manual_seed(7)
+    return [torch.randn(c, r, k, generator=g).to(torch.bfloat16) for c, r, k in shapes]
+
+
+def _grads(shapes, rank, step):
+    g = torch.Generator().manual_seed(1000 * step + rank + 1)
+    return [torch.randn(c, r, k, generator=g) * (1 + rank) for c, r, k in shapes]
+
+
+def _rank_main(rank, world, port, variant, buckets, steps, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from muon_newton_schulz_05_b200.sharded import ShardedMuon
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        opt = ShardedMuon(SHAPES, torch.bfloat16, torch.float32, variant=variant,
+                          buckets=buckets, ema=(variant == "anvil"),
+                          step_fn=_oracle_step_fn(variant), workspace_fn=lambda shapes: None)
+        params = _params(SHAPES)
+        hp = _hparams(variant)
+        for s in range(steps):
+            opt.step(params, _grads(SHAPES, rank, s), hp)
+        res = {"params": [p.float().numpy() for p in params]}
+        if variant == "anvil":
+            ema = [torch.zeros(c, r, k) for c, r, k in SHAPES]
+            opt.gather_ema(ema)
+            res["ema"] = [e.numpy() for e in ema]
+        out[rank] = res
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def _single_process(variant, steps, world):
+    """Every matrix stepped by one process on the mean of the ranks' gradients."""
+    from muon_newton_schulz_05_b200 import Bank
+    params = _params(SHAPES)
+    mom = [torch.zeros(c, r, k) for c, r, k in SHAPES]
+    slow = [torch.zeros(c, r, k) for c, r, k in SHAPES] if variant == "anvil" else [None] * 3
+    ema = [p.float().clone() for p in params] if variant == "anvil" else [None] * 3
+    step = _oracle_step_fn(variant)
+    hp = _hparams(variant)
+    for s in range(steps):
+        gs = [_grads(SHAPES, r, s) for r in range(world)]
+        mean = [(gs[0][b] + gs[1][b]) / world for b in range(len(SHAPES))]
+        step([Bank(params[b], mean[b], mom[b], slow[b], ema[b]) for b in range(len(SHAPES))],
+             hp, None)
+    return params, ema
+
+
+def _run(variant, buckets, steps=2, world=2):
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_rank_main, args=(world, port, variant, buckets, steps, out), nprocs=world,
+                 join=True)
+        return dict(out)
+
+
+@pytest.mark.parametrize("variant,buckets", [("muon", None), ("muon", [[0], [1, 2]]),
+                                             ("anvil", [[2], [0, 1]])])
+def test_sharded_step_equals_single_process_step(variant, buckets):
+    res = _run(variant, buckets)
+    ref_params, ref_ema = _single_process(variant, 2, 2)
+    for b in range(len(SHAPES)):
+        want = ref_params[b].float().numpy()
+        for r in (0, 1):
+            np.testing.assert_array_equal(res[r]["params"][b], want)
+        if variant == "anvil":
+            for r in (0, 1):
+                np.testing.assert_array_equal(res[r]["ema"][b], ref_ema[b].numpy())
+    # the step moved every matrix
+    p0 = _params(SHAPES)
+    for b in range(len(SHAPES)):
+        assert np.all(np.abs(res[0]["params"][b] - p0[b].float().numpy()).reshape(
+            SHAPES[b][0], -1).max(axis=1) > 0)
+
+
+def test_plan_owns_every_matrix_once_and_balances_gpt_bank():
+    for world in (1, 2, 4, 8):
+        plan = ShardPlan.build(GPT_SHAPES, world)
+        for b, (count, rows, cols) in enumerate(GPT_SHAPES):
+            got = sorted(i for r in range(world) for i in plan.buckets[0].owned[r][b])
+            assert got == list(range(count))
+        total = sum(c * ns_work(r, k) for c, r, k in GPT_SHAPES)
+        assert abs(sum(plan.load) - total) < 1e-6 * total
+        # 72 matrices of two weights: greedy lands within one small matrix of even
+        assert max(plan.load) - total / world <= ns_work(768, 768) + 1e-6 * total
+
+
+def test_plan_segments_aligned_and_pack_roundtrip():
+    plan = ShardPlan.build(SHAPES, 3, [[1], [0, 2]])
+    ts = [torch.arange(c * r * k, dtype=torch.float32).view(c, r, k) + 1000 * i
+          for i, (c, r, k) in enumerate(SHAPES)]
+    for k, bk in enumerate(plan.buckets):
+        for r in range(3):
+            assert all(o % 128 == 0 for o in bk.offsets[r])
+            used = [len(o) * SHAPES[b][1] * SHAPES[b][2] for o, b in zip(bk.owned[r], bk.banks)]
+            assert bk.offsets[r][-1] + used[-1] <= bk.seg
+        flat = torch.full((3 * bk.seg,), -1.0)
+        plan.pack(k, ts, flat)
+        back = [torch.zeros_like(t) for t in ts]
+        plan.unpack(k, flat, back)
+        for b in bk.banks:
+            assert torch.equal(back[b], ts[b])
+
+
+def test_plan_rejects_bad_buckets():
+    with pytest.raises(ValueError):
+        ShardPlan.build(SHAPES, 2, [[0], [1]])
+    with pytest.raises(ValueError):
+        ShardPlan.build(SHAPES, 2, [[0, 1], [1, 2]])
+    with pytest.raises(ValueError):
+        ShardPlan.build(SHAPES, 0)
