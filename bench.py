@@ -30,13 +30,19 @@ sys.path.insert(0, ROOT)
 METRIC = "Muon steps/s on GPT-124M matrix bank; NS TFLOP/s as % bf16 tensor peak"
 UNIT = "steps/s"
 WORKLOAD_ID = 2
-# kernel launches per step: momentum+norm, norm finalize, the Newton-Schulz
-# chain (one persistent launch), update
-LAUNCHES_PER_STEP = 4
 # DRAM bytes (read + write) of one Newton-Schulz chain launch on this workload,
 # from the ncu capture summarised in profiles/ns_gemm_gpt124m_bank.md. Set to
 # None whenever ns_gemm_kernel changes until it is captured again.
-NS_CHAIN_DRAM_BYTES = 5.889017e9
+NS_CHAIN_DRAM_BYTES = 6.020339e9
+
+
+def launches_per_step(w) -> int:
+    """Kernel launches of one optimizer step: momentum+norm, norm finalize and
+    the Newton-Schulz chain (one persistent launch, which also writes the
+    parameters of a Muon step on bf16 banks with rows a multiple of 8 long),
+    plus the update pass for every other bank (ANVIL, fp32, ragged rows)."""
+    fused = w.variant == "muon" and w.param_dtype == "bf16" and all(b.cols % 8 == 0 for b in w.banks)
+    return 3 if fused else 4
 
 
 def _args():
@@ -278,7 +284,8 @@ def run_native(args):
     step_fn = mb.anvil_step if anvil else mb.muon_step
     stream = torch.cuda.current_stream(dev)
     flops_step = _ns_flops(w)
-    launches_per_step = LAUNCHES_PER_STEP
+    n_launch = launches_per_step(w)
+    fused = n_launch == 3
 
     for _ in range(args.warmup):
         step_fn(banks, H, ws)
@@ -329,7 +336,8 @@ def run_native(args):
     pre_b = gsz + (16 if anvil else 8) + 4
     post_b = 2 + 2 * psz + (12 if anvil else 0)
     pre_gbs = elem_bytes * pre_b / (statistics.mean(pre_ms) * 1e-3) / 1e9
-    post_gbs = elem_bytes * post_b / (statistics.mean(post_ms) * 1e-3) / 1e9
+    # with the update fused into the chain's last step there is no update pass
+    post_gbs = None if fused else elem_bytes * post_b / (statistics.mean(post_ms) * 1e-3) / 1e9
 
     # -------- end to end through the public API with host buffers
     # Every step uploads its gradients from pinned host memory and reads the
@@ -410,16 +418,18 @@ def run_native(args):
             "traffic": NS_CHAIN_DRAM_BYTES if args.workload == WORKLOAD_ID else None,
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
                               "(profiles/ns_gemm_gpt124m_bank.md)",
-            "kernel": "ns_gemm_kernel (one persistent launch: 5 Newton-Schulz steps x "
-                      "Gram/Poly/Apply over the 72-matrix bank)",
+            "kernel": "ns_gemm_kernel (one persistent launch: every Newton-Schulz step x "
+                      "Gram/Poly/Apply over the bank" + (
+                          "; the last step's epilogue also writes the parameters)" if fused else ")"),
             "flops_per_launch": flops_step, "launch_ms": ns_avg_ms,
             "peak_kind": f"bf16 dense sustained, {peaks['src']}",
             "frac_of_burst": achieved / peaks["burst"],
         },
         "breakdown_ms": {"momentum_norm": statistics.mean(pre_ms), "ns_chain": ns_avg_ms,
-                         "update": statistics.mean(post_ms)},
+                         "update": None if fused else statistics.mean(post_ms),
+                         "after_chain": statistics.mean(post_ms)},
         "elementwise_gbs": {"momentum_norm": pre_gbs, "update": post_gbs, "peak": peaks["hbm"]},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * K,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": n_launch * K,
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)

@@ -62,11 +62,6 @@ __device__ __forceinline__ float round_store1(void* base, int dtype, long long i
   return x;
 }
 
-// value as stored (bf16 values are rounded to nearest even)
-__device__ __forceinline__ float stored(int dtype, float x) {
-  return dtype == MUON_BF16 ? __bfloat162float(__float2bfloat16_rn(x)) : x;
-}
-
 // U for one element; updates the momentum values in place.
 __device__ __forceinline__ float momentum_elem(const MomParams& p, float g, float& m, float& ms) {
   if (p.mode == kMomNone) return g;
@@ -198,11 +193,7 @@ cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total
 // ------------------------------------------------------------------ update
 __device__ __forceinline__ float update_elem(const UpdParams& p, const UpdBank& io, float th,
                                              float o, float ms) {
-  if (p.mode == kUpdCautious) {
-    const float mask = (o * ms > 0.0f) ? 1.0f : 0.0f;
-    return fmaf(-io.step_scale, o, fmaf(-p.lr_wd * mask, th, th));
-  }
-  return fmaf(-io.step_scale, o, th * (1.0f - p.lr_wd));
+  return param_update(p.mode, th, o, ms, io.step_scale, p.lr_wd);
 }
 
 __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ UpdParams p) {
@@ -211,6 +202,7 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
   for (int b = 0; b < p.nbanks; ++b) {
     const BankPlan& bp = p.bank[b];
     const UpdBank& io = p.io[b];
+    if (!io.param) continue;  // updated by the last Newton-Schulz step
     const long long per = static_cast<long long>(bp.R) * bp.C;
     const long long n = per * bp.count;
     const __nv_bfloat16* hi = bp.hi[p.final_buf];
@@ -269,7 +261,7 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
             float em[8];
             load8(io.ema, MUON_F32, e[u], em);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) em[t] = fmaf(p.ema_beta, em[t], (1.0f - p.ema_beta) * th[u][t]);
+            for (int t = 0; t < 8; ++t) em[t] = ema_elem(p.ema_beta, em[t], th[u][t]);
             store8(io.ema, MUON_F32, e[u], em);
           }
         }
@@ -303,7 +295,7 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
           float em[8];
           load8(io.ema, MUON_F32, e, em);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) em[t] = fmaf(p.ema_beta, em[t], (1.0f - p.ema_beta) * th[t]);
+          for (int t = 0; t < 8; ++t) em[t] = ema_elem(p.ema_beta, em[t], th[t]);
           store8(io.ema, MUON_F32, e, em);
         }
       }
@@ -322,7 +314,7 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
         const float th = load1(io.param, io.param_dtype, e);
         const float ms = p.mode == kUpdCautious ? io.mom_slow[e] : 0.0f;
         const float tn = round_store1(io.param, io.param_dtype, e, update_elem(p, io, th, o, ms));
-        if (io.ema) io.ema[e] = fmaf(p.ema_beta, io.ema[e], (1.0f - p.ema_beta) * tn);
+        if (io.ema) io.ema[e] = ema_elem(p.ema_beta, io.ema[e], tn);
       }
     }
   }
@@ -341,7 +333,7 @@ __global__ void __launch_bounds__(256) ema_kernel(float* ema, const void* param,
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long nthr = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = tid; i < n; i += nthr)
-    ema[i] = fmaf(beta, ema[i], (1.0f - beta) * load1(param, dtype, i));
+    ema[i] = ema_elem(beta, ema[i], load1(param, dtype, i));
 }
 
 __global__ void __launch_bounds__(256) blend_kernel(const void* theta, int tdtype, const float* ema,

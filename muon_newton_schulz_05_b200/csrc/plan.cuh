@@ -14,6 +14,7 @@
 #include <stdint.h>
 
 #include "muon_b200.h"
+#include "update_math.cuh"
 
 namespace muon {
 
@@ -70,6 +71,15 @@ struct BankPlan {
   float* part;                  // fp32 Gram partials [count][tiles_sym][ksplit][256][256]
 };
 
+// Parameter write of one bank (update pass, or fused into the chain's last step).
+struct UpdBank {
+  void* param;          // param (or O output in kUpdWriteO); nullptr: bank not handled here
+  int param_dtype;
+  const float* mom_slow;
+  float* ema;
+  float step_scale;     // lr * max(1, R/C)^(1/2)
+};
+
 // ---------------------------------------------------------------- GEMM chain
 // One persistent launch runs every Newton-Schulz step of every matrix. Tiles
 // are listed step by step, phase by phase (Gram, Reduce, Poly, Apply), bank by
@@ -95,6 +105,13 @@ struct NsGemmParams {
   int* status;                          // device status word
   unsigned long long wait_limit_ns;
   int fault;                            // test hook (muon_set_debug)
+  // parameter update fused into the last step's Apply epilogue (muon_step,
+  // anvil_step on banks whose rows are a multiple of 8 elements long):
+  // upd[b].param == nullptr leaves bank b to the update pass
+  UpdBank upd[MUON_MAX_BANKS];
+  int upd_mode;                         // kUpdDecoupled or kUpdCautious
+  float lr_wd;                          // lr * weight_decay
+  float ema_beta;
 };
 
 // ---------------------------------------------------------- momentum + norm
@@ -122,15 +139,6 @@ struct MomParams {
 };
 
 // --------------------------------------------------------------- update pass
-enum UpdMode : int { kUpdDecoupled = 0, kUpdCautious = 1, kUpdWriteO = 2 };
-
-struct UpdBank {
-  void* param;          // param (or O output in kUpdWriteO)
-  int param_dtype;
-  const float* mom_slow;
-  float* ema;
-  float step_scale;     // lr * max(1, R/C)^(1/2)
-};
 
 struct UpdParams {
   BankPlan bank[MUON_MAX_BANKS];
