@@ -141,7 +141,7 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   } else if (T.phase == kPoly) {
     if (bp.ksplit > 1) {
       T.dep_cnt = cnt + kReduce;
-      T.dep_target = kTileParts * bp.tiles_red * (T.iter + 1);
+      T.dep_target = kRedParts * bp.tiles_red * (T.iter + 1);
     } else {
       T.dep_cnt = cnt + kGram;
       T.dep_target = kTileParts * bp.tiles_sym * (T.iter + 1);
@@ -521,8 +521,9 @@ __device__ __forceinline__ bool epi_reduce(const NsGemmParams& p, EpiRing& e, co
   const int prow0 = (T.mat * bp.tiles_sym + T.sym_t) * ks * kTile + kBM * rank + 32 * q;
   const int pcol = half * 128 + kEpiCols * T.sub;
   const CUtensorMap* pmap = &p.maps[T.bank][kPartE];
+  constexpr int kAhead = kEpiBufs - 1;  // partials in flight beyond the one being summed
   if (lane == 0) {
-    for (int s = 0; s < 2 && s < ks; ++s) {
+    for (int s = 0; s < kAhead && s < ks; ++s) {
       mbar_arrive_expect_tx(&e.bar[s], kEpiChunkBytes);
       tma_load_2d(e.base + s * kEpiChunkBytes, pmap, &e.bar[s], pcol, prow0 + s * kTile);
     }
@@ -531,13 +532,13 @@ __device__ __forceinline__ bool epi_reduce(const NsGemmParams& p, EpiRing& e, co
 #pragma unroll
   for (int t = 0; t < 32; ++t) acc[t] = 0.0f;
   for (int s = 0; s < ks; ++s) {
-    // partial s+2 goes to the buffer of partial s-1, which every lane has summed
+    // partial s+kAhead goes to the buffer of partial s-1, which every lane has summed
     fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0 && s + 2 < ks) {
-      const int slot = (s + 2) % kEpiBufs;
+    if (lane == 0 && s + kAhead < ks) {
+      const int slot = (s + kAhead) % kEpiBufs;
       mbar_arrive_expect_tx(&e.bar[slot], kEpiChunkBytes);
-      tma_load_2d(e.base + slot * kEpiChunkBytes, pmap, &e.bar[slot], pcol, prow0 + (s + 2) * kTile);
+      tma_load_2d(e.base + slot * kEpiChunkBytes, pmap, &e.bar[slot], pcol, prow0 + (s + kAhead) * kTile);
     }
     const int slot = s % kEpiBufs;
     const bool ok = mbar_wait(&e.bar[slot], (e.parity >> slot) & 1u, abort_flag, p.status,
@@ -554,6 +555,7 @@ __device__ __forceinline__ bool epi_reduce(const NsGemmParams& p, EpiRing& e, co
       acc[4 * g + 3] += v.w;
     }
   }
+  static_assert(kEpiBufs >= 2, "the Reduce loop keeps one partial in flight");
   __syncwarp();
   uint32_t bits[32];
 #pragma unroll
@@ -587,7 +589,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
-  uint64_t* epibar = done + 1;  // kEpiWarps x kEpiBufs
+  uint64_t* pub = done + 1;     // per accumulator: this CTA's epilogue warps have stored the tile
+  uint64_t* epibar = pub + 2;   // kEpiWarps x kEpiBufs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + kEpiWarps * kEpiBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -609,6 +612,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 2 * kEpiWarps);  // the leader's: both CTAs' epilogue warps
     }
     mbar_init(done, 1);
+    for (int a = 0; a < 2; ++a) mbar_init(&pub[a], kEpiWarps);
     for (int w = 0; w < kEpiWarps * kEpiBufs; ++w) mbar_init(&epibar[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -762,13 +766,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         prefetch_update_row(p, p.upd[T.bank], bp, T.mat, r0 + lane, cw);
         fetch_param_bf16(p.upd[T.bank], bp, T.mat, r0 + lane, cw, thn);
       }
-      // the epilogue's own TMA loads read the same finished phase as the MMAs
+      // the epilogue's own TMA loads read the same finished phase as the MMAs;
+      // the first kEpiBufs chunks of the tile are requested now, while its
+      // MMAs run (each tile ends with all of its stores complete, so every
+      // buffer is free); a later chunk reuses a buffer once its store has
+      // read it
       if (lane == 0 && loads) {
         if (!wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) ok = false;
-        else {
-          bulk_wait_read<1>();  // ring buffer of chunk e.chunk: its last store has read it
-          epi_issue_load(p, e, T, bp, r0, cw, e.chunk);
-        }
+        else
+          for (int j = 0; j < kChunks && j < kEpiBufs; ++j) epi_issue_load(p, e, T, bp, r0, cw + j * kEpiCols, e.chunk + j);
       }
       if (!__all_sync(0xffffffffu, ok)) break;
       // the tcgen05.ld below is warp-collective: leave only if the whole warp does
@@ -781,14 +787,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int j = 0; j < kChunks; ++j) {
         const uint32_t k = e.chunk;
         const int c0 = cw + j * kEpiCols;
-        if (lane == 0) {
-          if (loads && j + 1 < kChunks) {
-            bulk_wait_read<1>();  // buffer of chunk k+1 was last stored from by chunk k-2
-            epi_issue_load(p, e, T, bp, r0, c0 + kEpiCols, k + 1);
-          } else if (!loads) {
-            bulk_wait_read<kEpiBufs - 1>();  // buffer of chunk k was last stored from by chunk k-3
-          }
-        }
+        if (lane == 0 && !loads) bulk_wait_read<kEpiBufs - 1>();  // buffer of chunk k: its store has read it
         __syncwarp();
         uint4 thc[4];
         if (fused) {
@@ -817,6 +816,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             epi_sym(T, bp, buf, lane, mirror, r);
           epi_store(p, T, bp, buf, r0, c0, lane, mirror);
         }
+        if (loads && j + kEpiBufs < kChunks) {
+          // chunk j's buffer takes chunk j + kEpiBufs once its store has read it
+          __syncwarp();
+          if (lane == 0) {
+            bulk_wait_read<0>();
+            epi_issue_load(p, e, T, bp, r0, c0 + kEpiBufs * kEpiCols, k + kEpiBufs);
+          }
+        }
         e.chunk = k + 1;
       }
       if (!ok) break;
@@ -824,12 +831,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
-        // this warp's part of the tile is in global memory: publish it
+        // this warp's part of the tile is in global memory
         bulk_wait_all();
         fence_proxy_async_global();
-        red_release_gpu_add(T.done_cnt, 1);
+        mbar_arrive(&pub[acc]);
+        // the CTA's part is complete once every epilogue warp's is: the first
+        // epilogue warp publishes it (one release per CTA and tile)
+        if (ew == 0) {
+          if (mbar_wait(&pub[acc], acc_phase, abort_flag, p.status, limit))
+            red_release_gpu_add(T.done_cnt, 1);
+          else
+            ok = false;
+        }
       }
-      __syncwarp();
+      ok = __shfl_sync(0xffffffffu, ok, 0);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }

@@ -23,7 +23,7 @@ constexpr int kTile = 256;         // GEMM tile (rows and cols) computed by one 
 constexpr int kBM = 128;           // tile rows held by one CTA of the pair
 constexpr int kBN = 256;           // tile cols (UMMA N); each CTA loads kBN/2 of B
 constexpr int kBK = 64;            // K per pipeline stage (one 128-byte swizzle row)
-constexpr int kStages = 4;         // TMA -> MMA pipeline depth (4..7 measured equal)
+constexpr int kStages = 4;         // TMA -> MMA pipeline depth (3 measured slower)
 constexpr int kATileBytes = kBM * kBK * 2;
 constexpr int kBTileBytes = (kBN / 2) * kBK * 2;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
@@ -32,7 +32,7 @@ constexpr int kEpiRows = 32;       // epilogue chunk: 32 rows x 32 columns per w
 constexpr int kEpiCols = 32;
 constexpr int kEpiHalfBytes = kEpiRows * kEpiCols * 2;      // one bf16 chunk
 constexpr int kEpiChunkBytes = 2 * kEpiHalfBytes;           // hi + lo, or out + mirror
-constexpr int kEpiBufs = 3;                                 // ring of chunk buffers per warp
+constexpr int kEpiBufs = 3;                                 // chunk buffers per warp
 constexpr int kEpiBufBytes = kEpiBufs * kEpiChunkBytes;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 1024 + 512;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, then epilogue
@@ -84,12 +84,14 @@ struct UpdBank {
 // One persistent launch runs every Newton-Schulz step of every matrix. Tiles
 // are listed step by step, phase by phase (Gram, Reduce, Poly, Apply), bank by
 // bank, matrix by matrix; CTA pairs take them round-robin. A tile waits on
-// per-matrix counters for the phase it reads; every epilogue warp of both
-// CTAs adds 1 to its own phase's counter when its stores are complete
-// (kTileParts per tile). Banks whose Gram K is much longer than the matrix is
+// per-matrix counters for the phase it reads. When all eight epilogue warps
+// of a CTA have stored their part of an MMA tile, one thread of the CTA adds
+// 1 to the tile's phase counter (kTileParts per tile); a Reduce sub-tile is
+// published by every epilogue warp of both CTAs (kRedParts). Banks whose Gram K is much longer than the matrix is
 // wide split that product along K: the split tiles store fp32 partials and
 // Reduce sub-tiles sum them into A.
-constexpr int kTileParts = 2 * kEpiWarps;
+constexpr int kTileParts = 2;                // MMA tiles: one part per CTA of the pair
+constexpr int kRedParts = 2 * kEpiWarps;     // Reduce sub-tiles: one per epilogue warp of both CTAs
 
 struct NsGemmParams {
   CUtensorMap maps[MUON_MAX_BANKS][kMaxMaps];
