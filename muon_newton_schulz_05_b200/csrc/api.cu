@@ -205,8 +205,7 @@ muon_status encode_map(CUtensorMap* m, void* ptr, int64_t inner, int64_t outer, 
 muon_status encode_bank_maps(const BankPlan& p, CUtensorMap* maps) {
   const int64_t rows = static_cast<int64_t>(p.count) * p.Rp;
   const int64_t srows = static_cast<int64_t>(p.count) * p.rp;
-  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B, sw64 = CU_TENSOR_MAP_SWIZZLE_64B,
-                           none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B, sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
   struct Spec {
     int slot;
     void* ptr;
@@ -221,9 +220,9 @@ muon_status encode_bank_maps(const BankPlan& p, CUtensorMap* maps) {
       {kHiE1, p.hi[1], p.Cp, rows, kEpiCols, kEpiRows, sw64},
       {kLoE, p.lo, p.Cp, rows, kEpiCols, kEpiRows, sw64},
       {kAE, p.A, p.rp, srows, kEpiCols, kEpiRows, sw64},
-      {kAT, p.A, p.rp, srows, kEpiRows, kEpiCols, none},
+      {kAMN, p.A, p.rp, srows, 64, 64, sw},
       {kBE, p.B, p.rp, srows, kEpiCols, kEpiRows, sw64},
-      {kBT, p.B, p.rp, srows, kEpiRows, kEpiCols, none},
+      {kBMN, p.B, p.rp, srows, 64, 64, sw},
   };
   for (const Spec& sp : specs) {
     muon_status st = encode_map(&maps[sp.slot], sp.ptr, sp.inner, sp.outer, sp.bi, sp.bo, sp.swz);

@@ -2,8 +2,11 @@
 //
 // One persistent launch runs the whole chain: every step and phase of every
 // matrix of every bank (see NsGemmParams). The three phases of a step are
-//   Gram : A = X X^T            (tall: A = Y^T Y)      upper tiles only, mirrored
-//   Poly : B = b A + c A A      (A symmetric)          upper tiles only, mirrored
+//   Gram : A = X X^T            (tall: A = Y^T Y)      upper 256-blocks only
+//   Poly : B = b A + c A A      (A symmetric)          upper 256-blocks only
+// A and B keep only their upper 256 x 256 blocks (diagonal blocks whole); an
+// operand block below the diagonal is read from the stored block across it,
+// as an MN-major (transposed) operand.
 //   Apply: X <- a X + B X       (tall: Y <- a Y + Y B) full tiles
 // ("Muonとは" / "Muonが登場": approximate orthogonalisation by Newton-Schulz
 // iteration, bf16 operands; the polynomial step is the method statement's).
@@ -39,6 +42,8 @@ struct Tile {
   float a, b, c;              // this step's coefficients
   int a_map, a_mn, a_base;
   int b_map, b_mn, b_base;
+  int a_sym, b_sym;           // operand is A or B: blocks below the diagonal read transposed
+  int a_tmap, b_tmap;         // the MN-major map for those blocks
   int* done_cnt;              // counter this tile's epilogue advances
   const int* dep_cnt;         // counter of the phase this tile reads
   int dep_target;             // value dep_cnt must reach first (0: nothing to wait for)
@@ -97,6 +102,8 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   T.split = 0;
   T.sub = 0;
   T.sym_t = 0;
+  T.a_sym = T.b_sym = 0;
+  T.a_tmap = T.b_tmap = 0;
   if (T.phase == kApply) {
     T.mat = local / bp.tiles_apply;
     const int t = local - T.mat * bp.tiles_apply;
@@ -173,17 +180,17 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
     T.a_mn = T.b_mn = 0;
     T.a_base = T.b_base = 0;
   } else if (T.phase == kPoly) {  // D[m][n] = sum_k A[m][k] A[n][k]
-    T.a_map = kAK; T.a_mn = 0; T.a_base = sbase;
-    T.b_map = kAK; T.b_mn = 0; T.b_base = sbase;
+    T.a_map = kAK; T.a_mn = 0; T.a_base = sbase; T.a_sym = 1; T.a_tmap = kAMN;
+    T.b_map = kAK; T.b_mn = 0; T.b_base = sbase; T.b_sym = 1; T.b_tmap = kAMN;
     T.nkb = bp.rp / kBK;
   } else {
     if (!bp.tall) {  // D[m][n] = sum_k B[m][k] X[k][n]
-      T.a_map = kBK_; T.a_mn = 0; T.a_base = sbase;
+      T.a_map = kBK_; T.a_mn = 0; T.a_base = sbase; T.a_sym = 1; T.a_tmap = kBMN;
       T.b_map = kHiMN0 + cur; T.b_mn = 1; T.b_base = xbase;
       T.nkb = bp.Rp / kBK;
     } else {         // D[m][n] = sum_k Y[m][k] B[n][k]
       T.a_map = kHiK0 + cur; T.a_mn = 0; T.a_base = xbase;
-      T.b_map = kBK_; T.b_mn = 0; T.b_base = sbase;
+      T.b_map = kBK_; T.b_mn = 0; T.b_base = sbase; T.b_sym = 1; T.b_tmap = kBMN;
       T.nkb = bp.Cp / kBK;
     }
   }
@@ -227,6 +234,13 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
   }
 }
 
+// Whether K block k0 of an operand whose rows start at mn0 is read
+// transposed: the operand is A or B and the 256-block (mn0, k0) lies below
+// the diagonal, so its values are those of the stored block (k0, mn0).
+__device__ __forceinline__ bool below_diagonal(int sym, int mn0, int k0) {
+  return sym && k0 / kTile < mn0 / kTile;
+}
+
 __device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_major, int ks) {
   return mn_major ? smem_desc_sw128(tile_addr + ks * 2048, 8192, 1024)
                   : smem_desc_sw128(tile_addr + ks * 32, 16, 1024);
@@ -235,14 +249,12 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_majo
 // ---------------------------------------------------------------- epilogues
 // Each epilogue warp owns 32 accumulator rows and 128 of the 256 columns and
 // works through them in 32 x 32 chunks. Global traffic goes through TMA only,
-// through a ring of kEpiBufs chunk buffers per warp: while chunk j is being
-// computed, the bulk load of chunk j+1's inputs (Apply: hi and lo of the
-// iterate; Poly: A) is in flight, and the stores of earlier chunks drain.
-// Row-wise halves use the 64-byte swizzle of the TMA box (16-byte group g of
+// through kEpiBufs chunk buffers per warp: the bulk loads of a tile's first
+// chunks (Apply: hi and lo of the iterate; Poly: A) are issued when the tile
+// starts, and the stores of earlier chunks drain while later ones are
+// computed. Halves use the 64-byte swizzle of the TMA box (16-byte group g of
 // row r at r*64 + ((g ^ ((r >> 1) & 3)) * 16)), so a lane reading or writing
-// its own row touches 8 distinct bank groups per quarter warp. The transposed
-// mirror half of an off-diagonal Gram/Poly chunk is a plain [32][32] array
-// written one column (64 contiguous bytes across the warp) at a time.
+// its own row touches 8 distinct bank groups per quarter warp.
 __device__ __forceinline__ uint32_t swz64_off(int r, int g) {
   return static_cast<uint32_t>(r * 64 + ((g ^ ((r >> 1) & 3)) << 4));
 }
@@ -420,16 +432,14 @@ __device__ __forceinline__ void epi_apply_update(const NsGemmParams& p, const Ti
   }
 }
 
-// Gram (A = D, times s^2 at step 0) or Poly (B = b A + c D) for this lane's
-// row; the transposed copy goes to the mirror half when `mirror`.
+// Gram (A = D, times s^2 at step 0) or Poly (B = b A + c D) for this lane's row.
 __device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, uint8_t* buf, int lane,
-                                        bool mirror, const uint32_t (&r)[32]) {
+                                        const uint32_t (&r)[32]) {
   float scl = 1.0f;
   if (T.phase != kPoly && T.iter == 0) {  // Gram / Reduce of U: fold 1 / ||U||^2 in here
     const float s = bp.scale[T.mat];
     scl = s * s;
   }
-  unsigned short* mir = reinterpret_cast<unsigned short*>(buf + kEpiHalfBytes);
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     const uint32_t off = swz64_off(lane, g);
@@ -452,20 +462,13 @@ __device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, uint8
 #pragma unroll
     for (int h = 0; h < 4; ++h) pk[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
     *reinterpret_cast<uint4*>(buf + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    if (mirror) {
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        mir[(8 * g + 2 * h) * kEpiRows + lane] = static_cast<unsigned short>(pk[h] & 0xFFFFu);
-        mir[(8 * g + 2 * h + 1) * kEpiRows + lane] = static_cast<unsigned short>(pk[h] >> 16);
-      }
-    }
   }
 }
 
 // Bulk-store ring chunk k (lane 0, after every lane's writes are visible to
 // the async proxy) as one bulk group.
 __device__ __forceinline__ void epi_store(const NsGemmParams& p, const Tile& T, const BankPlan& bp,
-                                          uint8_t* buf, int r0, int c0, int lane, bool mirror) {
+                                          uint8_t* buf, int r0, int c0, int lane) {
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
@@ -479,8 +482,6 @@ __device__ __forceinline__ void epi_store(const NsGemmParams& p, const Tile& T, 
     } else {
       const int base = T.mat * bp.rp;
       tma_store_2d(&p.maps[T.bank][T.phase == kPoly ? kBE : kAE], buf, c0, base + r0);
-      if (mirror)
-        tma_store_2d(&p.maps[T.bank][T.phase == kPoly ? kBT : kAT], buf + kEpiHalfBytes, r0, base + c0);
     }
     bulk_commit();
   }
@@ -511,7 +512,7 @@ __device__ __forceinline__ void epi_partial(const NsGemmParams& p, const Tile& T
 
 // Reduce sub-tile: this warp sums the ksplit partials of its 32 x 32 chunk in
 // split order (deterministic), folds in 1/||U||^2 at step 0, and stores the
-// bf16 chunk of A and, off the diagonal, its mirror. Requires every earlier
+// bf16 chunk of A. Requires every earlier
 // bulk store of the warp to be complete (all ring buffers free). False if a
 // wait gave up.
 __device__ __forceinline__ bool epi_reduce(const NsGemmParams& p, EpiRing& e, const Tile& T,
@@ -561,11 +562,10 @@ __device__ __forceinline__ bool epi_reduce(const NsGemmParams& p, EpiRing& e, co
 #pragma unroll
   for (int t = 0; t < 32; ++t) bits[t] = __float_as_uint(acc[t]);
   uint8_t* buf = e.base;  // every load has been consumed
-  const bool mirror = T.n0 != T.m0;
   const int r0 = T.m0 + kBM * rank + 32 * q;
   const int c0 = T.n0 + half * 128 + kEpiCols * T.sub;
-  epi_sym(T, bp, buf, lane, mirror, bits);
-  epi_store(p, T, bp, buf, r0, c0, lane, mirror);
+  epi_sym(T, bp, buf, lane, bits);
+  epi_store(p, T, bp, buf, r0, c0, lane);
   return true;
 }
 
@@ -663,8 +663,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint32_t bar = full_leader + 8u * static_cast<uint32_t>(stage);
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
             const int k0 = (T.kb0 + kb) * kBK;
-            load_operand(st, amap, bar, T.a_mn, T.a_base, T.m0 + kBM * rank, k0);
-            load_operand(st + kATileBytes, bmap, bar, T.b_mn, T.b_base, T.n0 + (kBN / 2) * rank, k0);
+            const bool at = below_diagonal(T.a_sym, T.m0, k0);
+            const bool bt = below_diagonal(T.b_sym, T.n0, k0);
+            load_operand(st, at ? &p.maps[T.bank][T.a_tmap] : amap, bar, at ? 1 : T.a_mn, T.a_base,
+                         T.m0 + kBM * rank, k0);
+            load_operand(st + kATileBytes, bt ? &p.maps[T.bank][T.b_tmap] : bmap, bar, bt ? 1 : T.b_mn,
+                         T.b_base, T.n0 + (kBN / 2) * rank, k0);
             issued_parity[stage] = static_cast<int>(phase);
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -687,7 +691,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         for (int tile = pair; ok && tile < ntiles; tile += npairs) {
           const Tile T = decode_tile(p, tile);
           if (T.phase == kReduce) continue;
-          const uint32_t idesc = idesc_bf16(2 * kBM, kBN, T.a_mn, T.b_mn);
           if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, limit)) {
             ok = false;
             break;
@@ -702,10 +705,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             tc_fence_after();
             const uint32_t a_addr = smem_u32(tiles + stage * kStageBytes);
             const uint32_t b_addr = a_addr + kATileBytes;
+            // the producer's choice of orientation for this K block
+            const int k0 = (T.kb0 + kb) * kBK;
+            const int a_mn = below_diagonal(T.a_sym, T.m0, k0) ? 1 : T.a_mn;
+            const int b_mn = below_diagonal(T.b_sym, T.n0, k0) ? 1 : T.b_mn;
+            const uint32_t idesc = idesc_bf16(2 * kBM, kBN, a_mn, b_mn);
 #pragma unroll
             for (int ks = 0; ks < kBK / 16; ++ks) {
-              umma_bf16_pair(d_tmem, operand_desc(a_addr, T.a_mn, ks),
-                             operand_desc(b_addr, T.b_mn, ks), idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+              umma_bf16_pair(d_tmem, operand_desc(a_addr, a_mn, ks), operand_desc(b_addr, b_mn, ks),
+                             idesc, (kb > 0 || ks > 0) ? 1u : 0u);
             }
             umma_commit_pair(&empty[stage]);  // frees this stage in both CTAs
             if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -757,7 +765,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                        kBM * static_cast<int>(rank) + 32 * q;
       const int r0 = T.m0 + kBM * static_cast<int>(rank) + 32 * q;  // first row of this warp
       const int cw = T.n0 + half * 128;                              // first column of this warp
-      const bool mirror = T.phase != kApply && T.n0 != T.m0;
       const bool loads = T.phase != kGram;
       // last step of a bank whose parameter update is fused into this epilogue
       const bool fused = T.phase == kApply && T.iter + 1 == p.ns_steps && p.upd[T.bank].param != nullptr;
@@ -813,8 +820,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (T.phase == kApply)
             epi_apply(T, bp, buf, lane, r);
           else
-            epi_sym(T, bp, buf, lane, mirror, r);
-          epi_store(p, T, bp, buf, r0, c0, lane, mirror);
+            epi_sym(T, bp, buf, lane, r);
+          epi_store(p, T, bp, buf, r0, c0, lane);
         }
         if (loads && j + kEpiBufs < kChunks) {
           // chunk j's buffer takes chunk j + kEpiBufs once its store has read it

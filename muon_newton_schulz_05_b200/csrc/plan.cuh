@@ -31,7 +31,7 @@ constexpr int kEpiWarps = 8;       // two per TMEM lane quadrant
 constexpr int kEpiRows = 32;       // epilogue chunk: 32 rows x 32 columns per warp
 constexpr int kEpiCols = 32;
 constexpr int kEpiHalfBytes = kEpiRows * kEpiCols * 2;      // one bf16 chunk
-constexpr int kEpiChunkBytes = 2 * kEpiHalfBytes;           // hi + lo, or out + mirror
+constexpr int kEpiChunkBytes = 2 * kEpiHalfBytes;           // hi + lo (Apply)
 constexpr int kEpiBufs = 3;                                 // chunk buffers per warp
 constexpr int kEpiBufBytes = kEpiBufs * kEpiChunkBytes;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 1024 + 512;
@@ -44,12 +44,12 @@ constexpr int kRedSub = 4;         // reduce sub-tiles per 256 x 256 tile (32 co
 constexpr int kMaxSplit = 16;      // K splits of a Gram product
 
 // Tensor-map slots per bank. Operand maps (128-byte swizzle): K-major boxes
-// of 128 rows x 64 columns, MN-major boxes of 64 x 64. Epilogue maps: 32 x 32
-// chunks, 64-byte swizzle for row-wise chunks, unswizzled for the transposed
-// mirror chunks of A and B.
+// of 128 rows x 64 columns, MN-major boxes of 64 x 64 (the A and B ones read
+// a block below the diagonal from its stored transpose). Epilogue maps: 32 x
+// 32 chunks, 64-byte swizzle.
 enum MapSlot : int {
   kHiK0 = 0, kHiK1 = 1, kHiMN0 = 2, kHiMN1 = 3, kAK = 4, kBK_ = 5,
-  kHiE0 = 6, kHiE1 = 7, kLoE = 8, kAE = 9, kAT = 10, kBE = 11, kBT = 12,
+  kHiE0 = 6, kHiE1 = 7, kLoE = 8, kAE = 9, kAMN = 10, kBE = 11, kBMN = 12,
   kPartE = 13  // fp32 Gram partial tiles, 32 x 32 boxes, 128-byte swizzle
 };
 
@@ -63,8 +63,8 @@ struct BankPlan {
   int tiles_red;                // reduce sub-tiles (tiles_sym * kRedSub when split)
   __nv_bfloat16* hi[2];         // iterate, high bf16 part (ping-pong)
   __nv_bfloat16* lo;            // iterate, low bf16 part (in place)
-  __nv_bfloat16* A;             // Gram matrix, count x rp x rp
-  __nv_bfloat16* B;             // b A + c A^2, count x rp x rp
+  __nv_bfloat16* A;             // Gram matrix, count x rp x rp; upper 256-blocks only
+  __nv_bfloat16* B;             // b A + c A^2, count x rp x rp; upper 256-blocks only
   float* partial;               // count x chunks sums of squares
   float* scale;                 // count: 1 / (||U||_F + eps)
   int* counters;                // count x 4: finished tile parts of Gram, Poly, Apply, Reduce
