@@ -33,7 +33,7 @@ WORKLOAD_ID = 2
 # DRAM bytes (read + write) of one Newton-Schulz chain launch on this workload,
 # from the ncu capture summarised in profiles/ns_gemm_gpt124m_bank.md. Set to
 # None whenever ns_gemm_kernel changes until it is captured again.
-NS_CHAIN_DRAM_BYTES = None
+NS_CHAIN_DRAM_BYTES = 5.501808e9
 
 
 def launches_per_step(w) -> int:
