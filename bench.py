@@ -33,16 +33,13 @@ WORKLOAD_ID = 2
 # DRAM bytes (read + write) of one Newton-Schulz chain launch on this workload,
 # from the ncu capture summarised in profiles/ns_gemm_gpt124m_bank.md. Set to
 # None whenever ns_gemm_kernel changes until it is captured again.
-NS_CHAIN_DRAM_BYTES = 5.501808e9
+NS_CHAIN_DRAM_BYTES = 5.191235e9
 
 
 def launches_per_step(w) -> int:
-    """Kernel launches of one optimizer step: momentum+norm, norm finalize and
-    the Newton-Schulz chain (one persistent launch, which also writes the
-    parameters of a Muon step on bf16 banks with rows a multiple of 8 long),
-    plus the update pass for every other bank (ANVIL, fp32, ragged rows)."""
-    fused = w.variant == "muon" and w.param_dtype == "bf16" and all(b.cols % 8 == 0 for b in w.banks)
-    return 3 if fused else 4
+    """Kernel launches of one optimizer step: momentum+norm, norm finalize, the
+    Newton-Schulz chain (one persistent launch) and the update pass."""
+    return 4
 
 
 def _args():
@@ -285,7 +282,6 @@ def run_native(args):
     stream = torch.cuda.current_stream(dev)
     flops_step = _ns_flops(w)
     n_launch = launches_per_step(w)
-    fused = n_launch == 3
 
     for _ in range(args.warmup):
         step_fn(banks, H, ws)
@@ -336,8 +332,7 @@ def run_native(args):
     pre_b = gsz + (16 if anvil else 8) + 4
     post_b = 2 + 2 * psz + (12 if anvil else 0)
     pre_gbs = elem_bytes * pre_b / (statistics.mean(pre_ms) * 1e-3) / 1e9
-    # with the update fused into the chain's last step there is no update pass
-    post_gbs = None if fused else elem_bytes * post_b / (statistics.mean(post_ms) * 1e-3) / 1e9
+    post_gbs = elem_bytes * post_b / (statistics.mean(post_ms) * 1e-3) / 1e9
 
     # -------- end to end through the public API with host buffers
     # Every step uploads its gradients from pinned host memory and reads the
@@ -419,15 +414,13 @@ def run_native(args):
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
                               "(profiles/ns_gemm_gpt124m_bank.md)",
             "kernel": "ns_gemm_kernel (one persistent launch: every Newton-Schulz step x "
-                      "Gram/Poly/Apply over the bank" + (
-                          "; the last step's epilogue also writes the parameters)" if fused else ")"),
+                      "Gram/Poly/Apply over the bank)",
             "flops_per_launch": flops_step, "launch_ms": ns_avg_ms,
             "peak_kind": f"bf16 dense sustained, {peaks['src']}",
             "frac_of_burst": achieved / peaks["burst"],
         },
         "breakdown_ms": {"momentum_norm": statistics.mean(pre_ms), "ns_chain": ns_avg_ms,
-                         "update": None if fused else statistics.mean(post_ms),
-                         "after_chain": statistics.mean(post_ms)},
+                         "update": statistics.mean(post_ms)},
         "elementwise_gbs": {"momentum_norm": pre_gbs, "update": post_gbs, "peak": peaks["hbm"]},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": n_launch * K,
         "clocks": clk,

@@ -195,14 +195,6 @@ muon_status muon_set_ns_events(void* before_ns, void* after_ns);
  * reports MUON_ERR_TIMEOUT through muon_device_status (results invalid). */
 muon_status muon_set_debug(int32_t fault_mode, double wait_limit_seconds);
 
-/* Where the parameter write of muon_step runs, process-wide. enabled != 0
- * (default): in the epilogue of the last Newton-Schulz step for every bank
- * with bf16 params, no EMA and cols a multiple of 8; every other bank (and
- * every anvil_step bank) uses the separate update pass. 0: always the update
- * pass. Both give the same bits. The pages define no such choice: it exists
- * so that the two paths can be compared. */
-muon_status muon_set_update_fusion(int32_t enabled);
-
 #ifdef __cplusplus
 }
 #endif

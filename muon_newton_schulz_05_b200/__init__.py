@@ -35,7 +35,7 @@ STATUS_NAMES = {
 
 EXPORTED = ("muon_abi_version", "muon_status_string", "muon_workspace_size", "muon_step",
             "anvil_step", "muon_orthogonalize", "ema_update", "readout_blend",
-            "muon_device_status", "muon_set_debug", "muon_set_ns_events", "muon_set_update_fusion",
+            "muon_device_status", "muon_set_debug", "muon_set_ns_events",
             "muon_orthogonalize_static")
 
 
@@ -75,7 +75,6 @@ _sig = {
     "readout_blend": (_i32, [_vp, _i32, _vp, _vp, _i32, _i64, _f, _vp]),
     "muon_device_status": (_i32, [_vp, _sz, _vp, _i32]),
     "muon_set_debug": (_i32, [_i32, ctypes.c_double]),
-    "muon_set_update_fusion": (_i32, [_i32]),
     "muon_set_ns_events": (_i32, [_vp, _vp]),
     "muon_orthogonalize_static": (_i32, [_vp, _i32, _vp, _i32, _i64, _i64, _i64,
                                          ctypes.POINTER(CHparams), _vp]),
@@ -260,13 +259,6 @@ def set_debug(fault_mode: int = 0, wait_limit_seconds: float = 0.0) -> None:
     _check(_lib.muon_set_debug(fault_mode, wait_limit_seconds), "muon_set_debug")
 
 
-def set_update_fusion(enabled: bool) -> None:
-    """Parameter write of muon_step on bf16 banks without EMA (rows a multiple
-    of 8 long) in the last Newton-Schulz step's epilogue (True, the default),
-    or always in the separate update pass (False); same results."""
-    _check(_lib.muon_set_update_fusion(1 if enabled else 0), "muon_set_update_fusion")
-
-
 def set_ns_events(before, after) -> None:
     """The next step call records these torch.cuda.Events around its
     Newton-Schulz launches (instrumentation for the benchmark)."""
@@ -286,6 +278,5 @@ def loaded_library_path() -> str:
 
 __all__: List[str] = ["Bank", "Hparams", "MuonError", "workspace_size", "alloc_workspace",
                       "muon_step", "anvil_step", "orthogonalize", "ema_update", "readout_blend",
-                      "device_status", "set_debug", "set_ns_events", "set_update_fusion", "status_string",
-                      "abi_version",
+                      "device_status", "set_debug", "set_ns_events", "status_string", "abi_version",
                       "raw_library", "CBank", "CHparams", "EXPORTED", "F32", "BF16"]

@@ -20,7 +20,6 @@ namespace {
 struct DebugState {
   int fault = 0;
   double wait_limit_s = 2.0;
-  bool fuse_update = true;
 };
 DebugState g_debug;
 
@@ -251,16 +250,6 @@ UpdBank update_io(const muon_bank& b, const muon_hparams* hp) {
   return UpdBank{b.param, b.param_dtype, b.momentum_slow, b.ema, static_cast<float>(double(hp->lr) * s)};
 }
 
-// The last Newton-Schulz step writes the parameters itself for the plain
-// decoupled step on bf16 parameters whose rows are whole 16-byte groups (8
-// elements). The cautious mask, the EMA and fp32 parameters add loads that
-// the epilogue cannot hide; those banks, measured faster that way, keep the
-// update pass.
-bool fuse_update(Variant v, const muon_bank& b) {
-  return g_debug.fuse_update && v == Variant::kMuon && b.param_dtype == MUON_BF16 &&
-         b.ema == nullptr && b.cols % 8 == 0;
-}
-
 muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_hparams* hp,
                      void* ws, size_t ws_bytes, cudaStream_t stream, const OrthoIO* oio) {
   int sms = 0;
@@ -322,20 +311,6 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   if (ev_before && cudaEventRecord(ev_before, stream) != cudaSuccess) return MUON_ERR_CUDA;
   gp.ns_steps = hp->ns_steps;
   gp.keep_lo = v == Variant::kOrtho ? 1 : 0;
-  // the parameter update rides on the last step's Apply epilogue wherever the
-  // rows allow 16-byte accesses; other banks keep the update pass
-  gp.upd_mode = v == Variant::kAnvil ? kUpdCautious : kUpdDecoupled;
-  gp.lr_wd = hp->lr * hp->weight_decay;
-  gp.ema_beta = hp->ema_beta;
-  bool update_pass = false;
-  for (int b = 0; b < nbanks; ++b) {
-    if (fuse_update(v, banks[b])) {
-      gp.upd[b] = update_io(banks[b], hp);
-    } else {
-      gp.upd[b] = UpdBank{};
-      update_pass = true;
-    }
-  }
   for (int i = 0; i < 3 * hp->ns_steps; ++i) gp.coef[i] = hp->coeffs[i];
   int gram = 0, red = 0, sym = 0, app = 0;
   for (int b = 0; b < nbanks; ++b) {
@@ -364,21 +339,17 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   up.use_lo = v == Variant::kOrtho ? 1 : 0;
   up.lr_wd = hp->lr * hp->weight_decay;
   up.ema_beta = hp->ema_beta;
-  long long total = 0;
   for (int b = 0; b < nbanks; ++b) {
     up.bank[b] = plans[b];
     if (v == Variant::kOrtho) {
       up.io[b] = {oio->out, oio->out_dtype, nullptr, nullptr, 0.0f};
-    } else if (gp.upd[b].param) {
-      up.io[b] = UpdBank{};  // done by the chain
     } else {
       up.io[b] = update_io(banks[b], hp);
     }
-    up.elem_begin[b] = total;
-    total += static_cast<long long>(banks[b].count) * banks[b].rows * banks[b].cols;
+    up.block_begin[b] = mp.block_begin[b];
   }
-  up.elem_begin[nbanks] = total;
-  if (update_pass && launch_update(up, total, sms, stream) != cudaSuccess) return MUON_ERR_CUDA;
+  up.block_begin[nbanks] = mp.block_begin[nbanks];
+  if (launch_update(up, mp.block_begin[nbanks], stream) != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }
 
@@ -593,12 +564,6 @@ muon_status muon_set_ns_events(void* before_ns, void* after_ns) {
   std::lock_guard<std::mutex> lk(g_mu);
   g_ev_before = static_cast<cudaEvent_t>(before_ns);
   g_ev_after = static_cast<cudaEvent_t>(after_ns);
-  return MUON_OK;
-}
-
-muon_status muon_set_update_fusion(int32_t enabled) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  g_debug.fuse_update = enabled != 0;
   return MUON_OK;
 }
 

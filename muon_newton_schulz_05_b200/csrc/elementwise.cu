@@ -191,139 +191,85 @@ cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total
 }
 
 // ------------------------------------------------------------------ update
-__device__ __forceinline__ float update_elem(const UpdParams& p, const UpdBank& io, float th,
-                                             float o, float ms) {
-  return param_update(p.mode, th, o, ms, io.step_scale, p.lr_wd);
-}
-
+// One block per (matrix, kChunk padded elements), the momentum pass's grid;
+// each thread takes one group of 8 at a time, so few registers and a full
+// SM of resident blocks keep enough loads in flight for HBM (a grid-stride
+// version with two groups per thread reached about half of the bandwidth).
+template <int Mode>
 __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ UpdParams p) {
-  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long nthr = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (int b = 0; b < p.nbanks; ++b) {
-    const BankPlan& bp = p.bank[b];
-    const UpdBank& io = p.io[b];
-    if (!io.param) continue;  // updated by the last Newton-Schulz step
-    const long long per = static_cast<long long>(bp.R) * bp.C;
-    const long long n = per * bp.count;
-    const __nv_bfloat16* hi = bp.hi[p.final_buf];
-    const __nv_bfloat16* lo = bp.lo;
-    const long long padded = static_cast<long long>(bp.Rp) * bp.Cp;
-    const unsigned long long ngroups = static_cast<unsigned long long>(n / 8);
-    if ((bp.C & 7) == 0 && ngroups < (1ull << 32)) {
-      // groups of 8 consecutive elements of a row; 32-bit index arithmetic and
-      // two independent groups per thread per pass (all loads issued first)
-      const uint32_t ng = static_cast<uint32_t>(ngroups);
-      const uint32_t gpr = static_cast<uint32_t>(bp.C / 8);
-      const uint32_t R = static_cast<uint32_t>(bp.R);
-      const uint32_t t32 = static_cast<uint32_t>(tid), n32 = static_cast<uint32_t>(nthr);
-      for (uint32_t g0 = t32; g0 < ng; g0 += 2 * n32) {
-        long long e[2], off[2];
-        bool has[2];
+  const int blk = blockIdx.x;
+  int b = 0;
+  while (b + 1 < p.nbanks && blk >= p.block_begin[b + 1]) ++b;
+  const BankPlan& bp = p.bank[b];
+  const UpdBank& io = p.io[b];
+  const int local = blk - p.block_begin[b];
+  const int mat = local / bp.chunks;
+  const int chunk = local - mat * bp.chunks;
+  const long long padded = static_cast<long long>(bp.Rp) * bp.Cp;
+  const long long e0 = static_cast<long long>(chunk) * kChunk;
+  const long long e1 = min(e0 + kChunk, padded);
+  const __nv_bfloat16* hi = bp.hi[p.final_buf] + mat * padded;
+  const __nv_bfloat16* lo = bp.lo + mat * padded;
+  const long long ubase = static_cast<long long>(mat) * bp.R * bp.C;
+  const int R = bp.R, C = bp.C, Cp = bp.Cp;
+  if ((C & 7) == 0) {
+    for (long long e = e0 + threadIdx.x * 8; e < e1; e += 256 * 8) {
+      const int prow = static_cast<int>(e / Cp);
+      const int pcol = static_cast<int>(e - static_cast<long long>(prow) * Cp);
+      if (prow >= R || pcol >= C) continue;
+      const long long i = ubase + static_cast<long long>(prow) * C + pcol;
+      float o[8], th[8], ms[8];
+      load8(hi, MUON_BF16, e, o);
+      if (p.use_lo) {
+        float l8[8];
+        load8(lo, MUON_BF16, e, l8);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const uint32_t g = g0 + static_cast<uint32_t>(u) * n32;
-          has[u] = g < ng;
-          const uint32_t gg = has[u] ? g : g0;
-          const uint32_t row = gg / gpr;
-          const uint32_t col = (gg - row * gpr) * 8u;
-          const uint32_t mat = row / R;
-          const uint32_t r = row - mat * R;
-          e[u] = static_cast<long long>(gg) * 8;
-          off[u] = (static_cast<long long>(mat) * bp.Rp + r) * bp.Cp + col;
-        }
-        float o[2][8], th[2][8], ms[2][8];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (!has[u]) continue;
-          load8(hi, MUON_BF16, off[u], o[u]);
-          if (p.mode != kUpdWriteO) load8(io.param, io.param_dtype, e[u], th[u]);
-          if (p.mode == kUpdCautious) load8(io.mom_slow, MUON_F32, e[u], ms[u]);
-          if (p.use_lo) {
-            float l8[8];
-            load8(lo, MUON_BF16, off[u], l8);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) o[u][t] += l8[t];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (!has[u]) continue;
-          if (p.mode == kUpdWriteO) {
-            store8(io.param, io.param_dtype, e[u], o[u]);
-            continue;
-          }
-#pragma unroll
-          for (int t = 0; t < 8; ++t)
-            th[u][t] = stored(io.param_dtype,
-                              update_elem(p, io, th[u][t], o[u][t], p.mode == kUpdCautious ? ms[u][t] : 0.0f));
-          store8(io.param, io.param_dtype, e[u], th[u]);
-          if (io.ema) {
-            float em[8];
-            load8(io.ema, MUON_F32, e[u], em);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) em[t] = ema_elem(p.ema_beta, em[t], th[u][t]);
-            store8(io.ema, MUON_F32, e[u], em);
-          }
-        }
+        for (int t = 0; t < 8; ++t) o[t] += l8[t];
       }
-    } else if ((bp.C & 7) == 0) {
-      for (long long g = tid; g < n / 8; g += nthr) {  // banks beyond 2^35 elements
-        const long long e = g * 8;
-        const long long mat = e / per;
-        const long long rem = e - mat * per;
-        const long long row = rem / bp.C;
-        const long long off = mat * padded + row * bp.Cp + (rem - row * bp.C);
-        float o[8], th[8], ms[8];
-        load8(hi, MUON_BF16, off, o);
-        if (p.use_lo) {
-          float l8[8];
-          load8(lo, MUON_BF16, off, l8);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) o[t] += l8[t];
-        }
-        if (p.mode == kUpdWriteO) {
-          store8(io.param, io.param_dtype, e, o);
-          continue;
-        }
-        load8(io.param, io.param_dtype, e, th);
-        if (p.mode == kUpdCautious) load8(io.mom_slow, MUON_F32, e, ms);
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          th[t] = stored(io.param_dtype, update_elem(p, io, th[t], o[t], p.mode == kUpdCautious ? ms[t] : 0.0f));
-        store8(io.param, io.param_dtype, e, th);
-        if (io.ema) {
-          float em[8];
-          load8(io.ema, MUON_F32, e, em);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) em[t] = ema_elem(p.ema_beta, em[t], th[t]);
-          store8(io.ema, MUON_F32, e, em);
-        }
+      if (Mode == kUpdWriteO) {
+        store8(io.param, io.param_dtype, i, o);
+        continue;
       }
-    } else {
-      for (long long e = tid; e < n; e += nthr) {
-        const long long mat = e / per;
-        const long long rem = e - mat * per;
-        const long long row = rem / bp.C;
-        const long long col = rem - row * bp.C;
-        const long long off = mat * padded + row * bp.Cp + col;
-        const float o = __bfloat162float(hi[off]) + (p.use_lo ? __bfloat162float(lo[off]) : 0.0f);
-        if (p.mode == kUpdWriteO) {
-          round_store1(io.param, io.param_dtype, e, o);
-          continue;
-        }
-        const float th = load1(io.param, io.param_dtype, e);
-        const float ms = p.mode == kUpdCautious ? io.mom_slow[e] : 0.0f;
-        const float tn = round_store1(io.param, io.param_dtype, e, update_elem(p, io, th, o, ms));
-        if (io.ema) io.ema[e] = ema_elem(p.ema_beta, io.ema[e], tn);
+      load8(io.param, io.param_dtype, i, th);
+      if (Mode == kUpdCautious) load8(io.mom_slow, MUON_F32, i, ms);
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        th[t] = stored(io.param_dtype, param_update(Mode, th[t], o[t], ms[t], io.step_scale, p.lr_wd));
+      store8(io.param, io.param_dtype, i, th);
+      if (io.ema) {
+        float em[8];
+        load8(io.ema, MUON_F32, i, em);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) em[t] = ema_elem(p.ema_beta, em[t], th[t]);
+        store8(io.ema, MUON_F32, i, em);
       }
+    }
+  } else {
+    for (long long e = e0 + threadIdx.x; e < e1; e += 256) {
+      const int prow = static_cast<int>(e / Cp);
+      const int pcol = static_cast<int>(e - static_cast<long long>(prow) * Cp);
+      if (prow >= R || pcol >= C) continue;
+      const long long i = ubase + static_cast<long long>(prow) * C + pcol;
+      const float o = __bfloat162float(hi[e]) + (p.use_lo ? __bfloat162float(lo[e]) : 0.0f);
+      if (Mode == kUpdWriteO) {
+        round_store1(io.param, io.param_dtype, i, o);
+        continue;
+      }
+      const float th = load1(io.param, io.param_dtype, i);
+      const float ms = Mode == kUpdCautious ? io.mom_slow[i] : 0.0f;
+      const float tn = round_store1(io.param, io.param_dtype, i, param_update(Mode, th, o, ms, io.step_scale, p.lr_wd));
+      if (io.ema) io.ema[i] = ema_elem(p.ema_beta, io.ema[i], tn);
     }
   }
 }
 
-cudaError_t launch_update(const UpdParams& p, long long total_elems, int num_sms, cudaStream_t s) {
-  long long want = (total_elems / 16 + 255) / 256;  // two groups of 8 per thread per pass
-  int grid = static_cast<int>(want < 1 ? 1 : (want > 8LL * num_sms ? 8LL * num_sms : want));
-  update_kernel<<<grid, 256, 0, s>>>(p);
+cudaError_t launch_update(const UpdParams& p, int total_blocks, cudaStream_t s) {
+  if (p.mode == kUpdCautious)
+    update_kernel<kUpdCautious><<<total_blocks, 256, 0, s>>>(p);
+  else if (p.mode == kUpdWriteO)
+    update_kernel<kUpdWriteO><<<total_blocks, 256, 0, s>>>(p);
+  else
+    update_kernel<kUpdDecoupled><<<total_blocks, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -325,113 +325,6 @@ __device__ __forceinline__ void epi_apply(const Tile& T, const BankPlan& bp, uin
   }
 }
 
-// Last step with the parameter update fused in (muon_step / anvil_step): O is
-// x' rounded to bf16 (the value the update pass would read back), and this
-// lane's row of the chunk, columns col0 .. col0+31, of the parameter (and the
-// slow momentum and EMA, where present) is read and written directly with
-// 16-byte accesses. The bank's rows are a multiple of 8 elements long, so a
-// group of 8 columns is either wholly inside the matrix or wholly padding.
-__device__ __forceinline__ void fetch_param_bf16(const UpdBank& u, const BankPlan& bp, int mat, int row,
-                                                 int col0, uint4 (&v)[4]) {
-  if (u.param_dtype != MUON_BF16 || row >= bp.R) return;
-  const __nv_bfloat16* base = static_cast<const __nv_bfloat16*>(u.param) +
-                              (static_cast<long long>(mat) * bp.R + row) * bp.C;
-#pragma unroll
-  for (int g = 0; g < 4; ++g)
-    if (col0 + 8 * g < bp.C) v[g] = *reinterpret_cast<const uint4*>(base + col0 + 8 * g);
-}
-
-// At the start of a fused tile, while its MMAs still run: pull this lane's row
-// segment (128 columns) of the parameter, slow momentum and EMA into L2.
-__device__ __forceinline__ void prefetch_update_row(const NsGemmParams& p, const UpdBank& u,
-                                                    const BankPlan& bp, int mat, int row, int col0) {
-  if (row >= bp.R || col0 >= bp.C) return;
-  const long long i = (static_cast<long long>(mat) * bp.R + row) * bp.C + col0;
-  const int n = min(128, bp.C - col0);  // elements of the segment
-  const int pb = u.param_dtype == MUON_BF16 ? 2 : 4;
-  const char* prm = static_cast<const char*>(u.param) + i * pb;
-  for (int off = 0; off < n * pb; off += 128) prefetch_l2(prm + off);
-  if (p.upd_mode == kUpdCautious)
-    for (int off = 0; off < n * 4; off += 128) prefetch_l2(reinterpret_cast<const char*>(u.mom_slow + i) + off);
-  if (u.ema)
-    for (int off = 0; off < n * 4; off += 128) prefetch_l2(reinterpret_cast<const char*>(u.ema + i) + off);
-}
-
-__device__ __forceinline__ void load_f32x8(const float* base, long long i, float (&x)[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(base + i);
-  const float4 b = *reinterpret_cast<const float4*>(base + i + 4);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-
-__device__ __forceinline__ void store_f32x8(float* base, long long i, const float (&x)[8]) {
-  *reinterpret_cast<float4*>(base + i) = make_float4(x[0], x[1], x[2], x[3]);
-  *reinterpret_cast<float4*>(base + i + 4) = make_float4(x[4], x[5], x[6], x[7]);
-}
-
-__device__ __forceinline__ void epi_apply_update(const NsGemmParams& p, const Tile& T, const BankPlan& bp,
-                                                 const uint8_t* buf, int lane, const uint32_t (&r)[32],
-                                                 int row, int col0, const uint4 (&thb)[4]) {
-  const UpdBank& u = p.upd[T.bank];
-  if (row >= bp.R) return;
-  float alpha = T.a, beta = 1.0f;
-  if (T.iter == 0) {  // a one-step chain: the iterate holds U; X0 = s U
-    const float s = bp.scale[T.mat];
-    alpha *= s;
-    beta = s;
-  }
-  const long long rowbase = (static_cast<long long>(T.mat) * bp.R + row) * bp.C;
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const int col = col0 + 8 * g;
-    if (col >= bp.C) continue;
-    const uint32_t off = swz64_off(lane, g);
-    const uint4 h4 = *reinterpret_cast<const uint4*>(buf + off);
-    const uint4 l4 = *reinterpret_cast<const uint4*>(buf + kEpiHalfBytes + off);
-    const uint32_t hw[4] = {h4.x, h4.y, h4.z, h4.w};
-    const uint32_t lw[4] = {l4.x, l4.y, l4.z, l4.w};
-    float o[8];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float y0 = fmaf(alpha, bf16_lo_f(hw[h]) + bf16_lo_f(lw[h]), beta * __uint_as_float(r[8 * g + 2 * h]));
-      const float y1 = fmaf(alpha, bf16_hi_f(hw[h]) + bf16_hi_f(lw[h]), beta * __uint_as_float(r[8 * g + 2 * h + 1]));
-      const uint32_t ho = pack_bf16x2(y0, y1);
-      o[2 * h] = bf16_lo_f(ho);
-      o[2 * h + 1] = bf16_hi_f(ho);
-    }
-    const long long i = rowbase + col;
-    float th[8], ms[8];
-    if (u.param_dtype == MUON_BF16) {
-      const uint32_t tw[4] = {thb[g].x, thb[g].y, thb[g].z, thb[g].w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        th[2 * h] = bf16_lo_f(tw[h]);
-        th[2 * h + 1] = bf16_hi_f(tw[h]);
-      }
-    } else {
-      load_f32x8(static_cast<const float*>(u.param), i, th);
-    }
-    if (p.upd_mode == kUpdCautious) load_f32x8(u.mom_slow, i, ms);
-#pragma unroll
-    for (int t = 0; t < 8; ++t)
-      th[t] = stored(u.param_dtype, param_update(p.upd_mode, th[t], o[t], ms[t], u.step_scale, p.lr_wd));
-    if (u.param_dtype == MUON_BF16) {
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(u.param) + i) =
-          make_uint4(pack_bf16x2(th[0], th[1]), pack_bf16x2(th[2], th[3]), pack_bf16x2(th[4], th[5]),
-                     pack_bf16x2(th[6], th[7]));
-    } else {
-      store_f32x8(static_cast<float*>(u.param), i, th);
-    }
-    if (u.ema) {
-      float em[8];
-      load_f32x8(u.ema, i, em);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) em[t] = ema_elem(p.ema_beta, em[t], th[t]);
-      store_f32x8(u.ema, i, em);
-    }
-  }
-}
-
 // Gram (A = D, times s^2 at step 0) or Poly (B = b A + c D) for this lane's row.
 __device__ __forceinline__ void epi_sym(const Tile& T, const BankPlan& bp, uint8_t* buf, int lane,
                                         const uint32_t (&r)[32]) {
@@ -766,13 +659,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int r0 = T.m0 + kBM * static_cast<int>(rank) + 32 * q;  // first row of this warp
       const int cw = T.n0 + half * 128;                              // first column of this warp
       const bool loads = T.phase != kGram;
-      // last step of a bank whose parameter update is fused into this epilogue
-      const bool fused = T.phase == kApply && T.iter + 1 == p.ns_steps && p.upd[T.bank].param != nullptr;
-      uint4 thn[4];  // the parameter row segment of the next chunk (bf16), fetched ahead
-      if (fused) {
-        prefetch_update_row(p, p.upd[T.bank], bp, T.mat, r0 + lane, cw);
-        fetch_param_bf16(p.upd[T.bank], bp, T.mat, r0 + lane, cw, thn);
-      }
       // the epilogue's own TMA loads read the same finished phase as the MMAs;
       // the first kEpiBufs chunks of the tile are requested now, while its
       // MMAs run (each tile ends with all of its stores complete, so every
@@ -796,12 +682,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int c0 = cw + j * kEpiCols;
         if (lane == 0 && !loads) bulk_wait_read<kEpiBufs - 1>();  // buffer of chunk k: its store has read it
         __syncwarp();
-        uint4 thc[4];
-        if (fused) {
-#pragma unroll
-          for (int g = 0; g < 4; ++g) thc[g] = thn[g];
-          if (j + 1 < kChunks) fetch_param_bf16(p.upd[T.bank], bp, T.mat, r0 + lane, c0 + kEpiCols, thn);
-        }
         uint32_t r[32];
         tmem_ld32(tb + j * kEpiCols, r);
         if (loads && !epi_wait_load(p, e, k, abort_flag)) {
@@ -813,9 +693,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         uint8_t* buf = ring_buf(e, k);
         if (split) {
           epi_partial(p, T, buf, lane, prow, half * 128 + j * kEpiCols, r);
-        } else if (fused) {
-          epi_apply_update(p, T, bp, buf, lane, r, r0 + lane, c0, thc);
-          fence_proxy_async_smem();  // these reads precede the next bulk load into buf
         } else {
           if (T.phase == kApply)
             epi_apply(T, bp, buf, lane, r);

@@ -71,9 +71,9 @@ struct BankPlan {
   float* part;                  // fp32 Gram partials [count][tiles_sym][ksplit][256][256]
 };
 
-// Parameter write of one bank (update pass, or fused into the chain's last step).
+// Parameter write of one bank (the update pass).
 struct UpdBank {
-  void* param;          // param (or O output in kUpdWriteO); nullptr: bank not handled here
+  void* param;          // param (or O output in kUpdWriteO)
   int param_dtype;
   const float* mom_slow;
   float* ema;
@@ -107,13 +107,6 @@ struct NsGemmParams {
   int* status;                          // device status word
   unsigned long long wait_limit_ns;
   int fault;                            // test hook (muon_set_debug)
-  // parameter update fused into the last step's Apply epilogue (muon_step,
-  // anvil_step on banks whose rows are a multiple of 8 elements long):
-  // upd[b].param == nullptr leaves bank b to the update pass
-  UpdBank upd[MUON_MAX_BANKS];
-  int upd_mode;                         // kUpdDecoupled or kUpdCautious
-  float lr_wd;                          // lr * weight_decay
-  float ema_beta;
 };
 
 // ---------------------------------------------------------- momentum + norm
@@ -145,7 +138,7 @@ struct MomParams {
 struct UpdParams {
   BankPlan bank[MUON_MAX_BANKS];
   UpdBank io[MUON_MAX_BANKS];
-  long long elem_begin[MUON_MAX_BANKS + 1];   // logical elements, prefix sums
+  int block_begin[MUON_MAX_BANKS + 1];   // first block of each bank (the momentum pass's grid)
   int nbanks;
   int mode;
   int final_buf;        // hi buffer holding the last iterate
@@ -158,8 +151,7 @@ struct UpdParams {
 cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total_mats,
                                  cudaStream_t s);
 cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s);  // whole chain
-cudaError_t launch_update(const UpdParams& p, long long total_elems, int num_sms,
-                          cudaStream_t s);
+cudaError_t launch_update(const UpdParams& p, int total_blocks, cudaStream_t s);
 cudaError_t launch_ema(float* ema, const void* param, int param_dtype, long long n, float beta,
                        int num_sms, cudaStream_t s);
 cudaError_t launch_blend(const void* theta, int theta_dtype, const float* ema, void* out,

@@ -1,6 +1,5 @@
-// Element arithmetic of the parameter update, shared by the standalone update
-// pass and the update fused into the last Newton-Schulz step, so that both
-// give the same bits.
+// Element arithmetic of the parameter update (the update pass and the
+// standalone EMA).
 //   decoupled : theta <- theta (1 - lr wd) - lr s O         ("Muonとは")
 //   cautious  : theta <- theta - lr wd mask theta - lr s O,
 //               mask = [O M_slow > 0]                        ("ANVIL II와 가중치 평균")

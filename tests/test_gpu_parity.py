@@ -405,54 +405,3 @@ def test_transformer_2p5b_bank_sampled():
                                            oracle.shape_scale(R, C)) - t0
             ok, r = delta_ok(t0, f64(bk.param[i]), dref, "bf16")
             assert ok, ("delta", b, i, r)
-
-
-# ------------------------------------------ update fused into the last step
-# (count, rows, cols, param dtype, EMA): bf16 banks without EMA whose rows are a
-# multiple of 8 long take the fused write; the others take the update pass in
-# the same call
-FUSION_BANKS = [(3, 300, 512, torch.bfloat16, False), (2, 520, 264, torch.bfloat16, False),
-                (1, 768, 3072, torch.bfloat16, False), (2, 256, 768, torch.float32, False),
-                (1, 96, 1000, torch.bfloat16, True), (2, 64, 77, torch.bfloat16, False)]
-
-
-def test_fused_update_matches_update_pass_bitwise():
-    """The parameter write in the last Newton-Schulz epilogue and the separate
-    update pass give the same bits (param, momentum, EMA) over several steps."""
-    hp = dict(lr=0.03, mu=0.95, weight_decay=0.2, nesterov=True, coeffs=[QUINTIC] * 5, eps=1e-7,
-              ema_beta=0.9)
-    H = mb.Hparams.from_dict(hp)
-
-    def make():
-        banks = []
-        for i, (c, r, k, dt, ema) in enumerate(FUSION_BANKS):
-            th = mi.gaussian(c * r, k, seed=40 + i, sigma=0.02).reshape(c, r, k).to(dt).to(DEV)
-            banks.append(mb.Bank(th, None, torch.zeros(c, r, k, device=DEV), None,
-                                 th.float().clone() if ema else None))
-        return banks
-
-    runs = []
-    for fusion in (True, False):
-        mb.set_update_fusion(fusion)
-        try:
-            banks = make()
-            ws = mb.alloc_workspace([b.shape for b in banks])
-            for s in range(3):
-                for i, (b, spec) in enumerate(zip(banks, FUSION_BANKS)):
-                    c, r, k = spec[:3]
-                    b.grad = mi.gaussian(c * r, k, seed=700 + 10 * s + i, sigma=1.0).reshape(
-                        c, r, k).to(torch.bfloat16).to(DEV)
-                mb.muon_step(banks, H, ws)
-            assert mb.device_status(ws) == 0
-            runs.append(banks)
-        finally:
-            mb.set_update_fusion(True)
-    for a, b in zip(*runs):
-        assert torch.equal(a.param, b.param)
-        assert torch.equal(a.momentum, b.momentum)
-        if a.ema is not None:
-            assert torch.equal(a.ema, b.ema)
-    # and the step did move every matrix
-    fresh = make()
-    for a, f in zip(runs[0], fresh):
-        assert (a.param.float() - f.param.float()).abs().flatten(1).amax(1).min() > 0
