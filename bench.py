@@ -22,6 +22,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -204,7 +205,9 @@ class Clocks:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # raw samples go to a scratch file; their summary goes into the JSON line
+        self.path = os.path.join(os.environ.get("MUON_BENCH_CLOCKS_DIR", tempfile.gettempdir()),
+                                 f"muon_bench_clocks_rank{index}.csv")
 
     def start(self):
         try:
