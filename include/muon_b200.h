@@ -34,8 +34,9 @@
  *     non-OK status means nothing was launched. Faults found on the device
  *     (a bounded wait that ran out) are reported by muon_device_status.
  *   - Every device pointer must be 16-byte aligned. param, momentum,
- *     momentum_slow and ema are updated in place and must not overlap each
- *     other or the workspace; grad is read only.
+ *     momentum_slow and ema are updated in place and must not overlap one
+ *     another, in the same bank or in another bank of the call (checked:
+ *     MUON_ERR_ALIAS), nor the workspace (not checked); grad is read only.
  */
 #ifndef MUON_B200_H
 #define MUON_B200_H

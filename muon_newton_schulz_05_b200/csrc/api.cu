@@ -67,6 +67,9 @@ constexpr size_t kHeaderBytes = 4096;  // device status word at offset 0
 
 muon_status check_shape(int64_t count, int64_t rows, int64_t cols) {
   if (count < 1 || rows < 1 || cols < 1) return MUON_ERR_SHAPE;
+  // bound each factor first so that the products below cannot overflow
+  if (count >= (int64_t(1) << 31) || rows >= (int64_t(1) << 24) || cols >= (int64_t(1) << 24))
+    return MUON_ERR_SHAPE;
   const int64_t Rp = round_up(rows, kPad), Cp = round_up(cols, kPad);
   const int64_t rp = rows > cols ? Cp : Rp;
   // TMA coordinates and tile indices are 32-bit
@@ -99,6 +102,10 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 muon_status check_banks(const muon_bank* banks, int32_t nbanks, bool anvil) {
   if (!banks) return MUON_ERR_NULL;
   if (nbanks < 1 || nbanks > MUON_MAX_BANKS) return MUON_ERR_SHAPE;
+  // every buffer the step writes, over all banks: none may overlap another
+  const void* bufs[4 * MUON_MAX_BANKS];
+  size_t sz[4 * MUON_MAX_BANKS];
+  int nb = 0;
   for (int b = 0; b < nbanks; ++b) {
     const muon_bank& k = banks[b];
     muon_status st = check_shape(k.count, k.rows, k.cols);
@@ -110,13 +117,16 @@ muon_status check_banks(const muon_bank* banks, int32_t nbanks, bool anvil) {
         !aligned16(k.momentum_slow) || !aligned16(k.ema))
       return MUON_ERR_ALIGN;
     const size_t n = static_cast<size_t>(k.count * k.rows * k.cols);
-    const size_t np = n * (k.param_dtype == MUON_BF16 ? 2 : 4);
-    const void* bufs[4] = {k.param, k.momentum, anvil ? k.momentum_slow : nullptr, k.ema};
-    const size_t sz[4] = {np, n * 4, n * 4, n * 4};
-    for (int i = 0; i < 4; ++i)
-      for (int j = i + 1; j < 4; ++j)
-        if (overlap(bufs[i], sz[i], bufs[j], sz[j])) return MUON_ERR_ALIAS;
+    const void* w[4] = {k.param, k.momentum, anvil ? k.momentum_slow : nullptr, k.ema};
+    const size_t wz[4] = {n * (k.param_dtype == MUON_BF16 ? 2 : 4), n * 4, n * 4, n * 4};
+    for (int i = 0; i < 4; ++i) {
+      bufs[nb] = w[i];
+      sz[nb++] = wz[i];
+    }
   }
+  for (int i = 0; i < nb; ++i)
+    for (int j = i + 1; j < nb; ++j)
+      if (overlap(bufs[i], sz[i], bufs[j], sz[j])) return MUON_ERR_ALIAS;
   return MUON_OK;
 }
 

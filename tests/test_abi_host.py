@@ -134,6 +134,42 @@ def test_validation_paths(fn):
         assert _call(fn, _bank(ema=FAKE + 0x4000), hp=mb.Hparams(ema_beta=1.0)) == 5
 
 
+@pytest.mark.parametrize("fn", ["muon_step", "anvil_step"])
+def test_huge_shapes_rejected_without_overflow(fn):
+    ok = dict(momentum_slow=FAKE + 0x3000 if fn == "anvil_step" else None)
+    for kw in (dict(count=1 << 62), dict(rows=1 << 40), dict(cols=1 << 40),
+               dict(count=1 << 30, rows=1 << 23, cols=1 << 23)):
+        assert _call(fn, _bank(**kw, **ok)) == 2, kw
+
+
+@pytest.mark.parametrize("fn", ["muon_step", "anvil_step"])
+def test_buffers_of_different_banks_must_not_overlap(fn):
+    """A buffer a step writes may not overlap one of another bank either."""
+    lib = mb.raw_library()
+    h = mb.Hparams().to_c()
+    anvil = fn == "anvil_step"
+
+    def bank(base):
+        return _bank(param=base, grad=base + 0x1000, momentum=base + 0x2000,
+                     momentum_slow=base + 0x3000 if anvil else None)
+
+    def call(b0, b1):
+        arr = (mb.CBank * 2)(b0, b1)
+        return getattr(lib, fn)(arr, 2, ctypes.byref(h), FAKE * 16, 1 << 30, None)
+
+    import torch
+    if not torch.cuda.is_available():
+        # valid arguments get past validation (and then fail on the missing
+        # GPU); never run where kernels would launch on these fake addresses
+        assert call(bank(FAKE), bank(FAKE + 0x8000)) == 7
+    b1 = bank(FAKE + 0x8000)
+    b1.momentum = FAKE  # bank 1's momentum on bank 0's parameters
+    assert call(bank(FAKE), b1) == 9
+    b1 = bank(FAKE + 0x8000)
+    b1.param = FAKE + 0x2000 + 64  # inside bank 0's momentum
+    assert call(bank(FAKE), b1) == 9
+
+
 def test_valid_call_without_gpu_reports_cuda_error():
     """All arguments valid: the first CUDA call fails cleanly on a CPU host."""
     import torch
