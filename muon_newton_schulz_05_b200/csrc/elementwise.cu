@@ -1,6 +1,7 @@
 // Bandwidth-bound passes of the step:
-//   momentum_norm : M <- mu M + (1 - mu) G, U (Nesterov or not; or the two
-//                   ANVIL momenta), writes U as the bf16 hi/lo iterate in the
+//   momentum_norm : M <- mu M + (1 - mu) G (or the SGD form M <- mu M + G),
+//                   U (Nesterov or not; or the two ANVIL momenta), writes U as
+//                   the bf16 hi/lo iterate in the
 //                   padded working layout and per-block partial sums of U^2
 //   norm_finalize : 1 / (||U||_F + eps) per matrix from the partials, in a
 //                   fixed order (deterministic); resets the matrix's

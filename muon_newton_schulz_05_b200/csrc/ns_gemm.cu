@@ -4,12 +4,12 @@
 // matrix of every bank (see NsGemmParams). The three phases of a step are
 //   Gram : A = X X^T            (tall: A = Y^T Y)      upper 256-blocks only
 //   Poly : B = b A + c A A      (A symmetric)          upper 256-blocks only
+//   Apply: X <- a X + B X       (tall: Y <- a Y + Y B) full tiles
 // A and B keep only their upper 256 x 256 blocks (diagonal blocks whole); an
 // operand block below the diagonal is read from the stored block across it,
 // as an MN-major (transposed) operand.
-//   Apply: X <- a X + B X       (tall: Y <- a Y + Y B) full tiles
 // ("Muonとは" / "Muonが登場": approximate orthogonalisation by Newton-Schulz
-// iteration, bf16 operands; the polynomial step is the method statement's).
+// iteration, bf16 operands; the polynomial step is the method statement's.)
 //
 // CTA pairs (clusters of 2 on one TPC) compute 256 x 256 output tiles with the
 // 2-SM MMA (tcgen05.mma.cta_group::2, M = 256, N = 256, K = 16): each CTA
@@ -18,13 +18,14 @@
 // No TMA multicast is used; only the MMA commits arrive on both CTAs.
 //
 // Block layout (320 threads, one block per SM), in both CTAs of a pair:
-//   warp 0     one thread issues this CTA's TMA loads into a 6-stage ring;
-//              completion is counted on the even (leader) CTA's barrier
+//   warp 0     one thread issues this CTA's TMA loads into a kStages-deep
+//              ring; completion is counted on the even (leader) CTA's barrier
 //   warp 1     allocates 512 TMEM columns (pair allocation); in the leader one
 //              thread issues the MMAs into one of two 256-column accumulators
 //   warps 2..9 epilogue: tcgen05.ld this CTA's 128 accumulator rows (warp w
 //              reads TMEM lanes 32*(w%4)..+31; two warps per lane quadrant
-//              split the 256 columns), apply the phase's axpy and store
+//              split the 256 columns), apply the phase's axpy and store;
+//              one thread per CTA publishes the finished tile
 // The epilogue of tile t overlaps the MMAs of tile t+1 through the two
 // accumulators. Every wait is bounded (muon::mbar_wait*).
 #include <cuda_runtime.h>
