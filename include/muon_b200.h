@@ -62,7 +62,9 @@ typedef enum {
   MUON_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than muon_workspace_size */
   MUON_ERR_CUDA = 7,        /* a CUDA runtime call failed (launch, attribute) */
   MUON_ERR_TIMEOUT = 8,     /* a bounded device-side wait ran out             */
-  MUON_ERR_ALIAS = 9        /* in-place buffers overlap                       */
+  MUON_ERR_ALIAS = 9,       /* in-place buffers overlap                       */
+  MUON_ERR_BOUNDS = 10      /* debug build only: an index outside its buffer
+                               (the access was skipped; results invalid)      */
 } muon_status;
 
 typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype;

@@ -14,11 +14,15 @@ from dataclasses import dataclass, field
 from typing import List, Optional, Sequence, Tuple
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmuonb200.so")
+# MUON_B200_CHECK=1 selects the debug build with device-side bounds checks
+# (`build.py --check`); the default is the release library.
+LIB_PATH = os.path.join(_PKG, "libmuonb200_check.so" if os.environ.get("MUON_B200_CHECK") == "1"
+                        else "libmuonb200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python muon_newton_schulz_05_b200/build.py` "
+        f"{LIB_PATH} is missing: build it with `python muon_newton_schulz_05_b200/build.py"
+        f"{' --check' if LIB_PATH.endswith('_check.so') else ''}` "
         "(this package has no fallback implementation)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -30,7 +34,7 @@ F32, BF16 = 0, 1
 STATUS_NAMES = {
     0: "MUON_OK", 1: "MUON_ERR_NULL", 2: "MUON_ERR_SHAPE", 3: "MUON_ERR_DTYPE",
     4: "MUON_ERR_ALIGN", 5: "MUON_ERR_HPARAM", 6: "MUON_ERR_WORKSPACE", 7: "MUON_ERR_CUDA",
-    8: "MUON_ERR_TIMEOUT", 9: "MUON_ERR_ALIAS",
+    8: "MUON_ERR_TIMEOUT", 9: "MUON_ERR_ALIAS", 10: "MUON_ERR_BOUNDS",
 }
 
 EXPORTED = ("muon_abi_version", "muon_status_string", "muon_workspace_size", "muon_step",

@@ -1,6 +1,8 @@
 """Build libmuonb200.so in-tree with nvcc for sm_100a.
 
-Usage: python muon_newton_schulz_05_b200/build.py [--verbose-ptxas]
+Usage: python muon_newton_schulz_05_b200/build.py [--verbose-ptxas] [--check]
+(--check builds libmuonb200_check.so with device-side bounds checks, -DMUON_CHECK;
+the binding loads it instead when MUON_B200_CHECK=1)
 (run by path: the script does not import the package, so it works before
 the library exists)
 The CUDA runtime is linked statically; the driver entry point used for TMA
@@ -17,8 +19,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmuonb200.so")
+LIB_CHECK = os.path.join(PKG, "libmuonb200_check.so")
 SOURCES = ["api.cu", "elementwise.cu", "ns_gemm.cu"]
-HEADERS = ["plan.cuh", "ptx.cuh"]
+HEADERS = ["plan.cuh", "ptx.cuh", "update_math.cuh", "check.cuh"]
 
 
 def nvcc() -> str:
@@ -28,35 +31,37 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(INCLUDE, "muon_b200.h"))
     deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
+def build(force: bool = False, ptxas_verbose: bool = False, check: bool = False) -> str:
+    lib = LIB_CHECK if check else LIB
+    if not force and not needs_build(lib):
+        return lib
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
            "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared", "-cudart", "static",
-           "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp"]
+           "-I", INCLUDE, "-I", CSRC, "-o", lib + ".tmp"]
+    if check:
+        cmd += ["-DMUON_CHECK"]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libmuonb200.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if ptxas_verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv)
-    print(LIB)
+    print(build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv, check="--check" in sys.argv))

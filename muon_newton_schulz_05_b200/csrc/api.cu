@@ -285,6 +285,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   mp.nesterov = hp->nesterov ? 1 : 0;
   mp.sgd = (v == Variant::kMuon && hp->sgd_momentum) ? 1 : 0;
   mp.eps = hp->eps;
+  mp.status = status;
   int blocks = 0, mats = 0;
   for (int b = 0; b < nbanks; ++b) {
     mp.bank[b] = plans[b];
@@ -349,6 +350,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   up.use_lo = v == Variant::kOrtho ? 1 : 0;
   up.lr_wd = hp->lr * hp->weight_decay;
   up.ema_beta = hp->ema_beta;
+  up.status = status;
   for (int b = 0; b < nbanks; ++b) {
     up.bank[b] = plans[b];
     if (v == Variant::kOrtho) {
@@ -400,6 +402,7 @@ const char* muon_status_string(muon_status s) {
     case MUON_ERR_CUDA: return "MUON_ERR_CUDA: CUDA runtime error";
     case MUON_ERR_TIMEOUT: return "MUON_ERR_TIMEOUT: a bounded device wait ran out";
     case MUON_ERR_ALIAS: return "MUON_ERR_ALIAS: in-place buffers overlap";
+    case MUON_ERR_BOUNDS: return "MUON_ERR_BOUNDS: an index outside its buffer (debug build)";
   }
   return "unknown muon_status";
 }

@@ -105,14 +105,18 @@ __global__ void __launch_bounds__(256) momentum_norm_kernel(const __grid_constan
   __nv_bfloat16* lo = bp.lo + mat * padded;
   const long long ubase = static_cast<long long>(mat) * bp.R * bp.C;
   const int R = bp.R, C = bp.C, Cp = bp.Cp;
+  // buffer extents for the debug build's checks: logical and padded elements
+  const long long nlog = static_cast<long long>(bp.count) * R * C;
+  const long long nwork = static_cast<long long>(bp.count) * padded;
+  const long long wbase = static_cast<long long>(mat) * padded;
   float ss = 0.0f;
   if ((C & 7) == 0) {
     for (long long e = e0 + threadIdx.x * 8; e < e1; e += 256 * 8) {
       const int prow = static_cast<int>(e / Cp);
       const int pcol = static_cast<int>(e - static_cast<long long>(prow) * Cp);
+      const long long i = ubase + static_cast<long long>(prow) * C + pcol;
       float u[8];
-      if (prow < R && pcol < C) {
-        const long long i = ubase + static_cast<long long>(prow) * C + pcol;
+      if (prow < R && pcol < C && in_bounds(i + 8 <= nlog, p.status)) {
         float g[8], m[8], ms[8];
         load8(io.grad, io.grad_dtype, i, g);
         if (p.mode != kMomNone) load8(io.mom, MUON_F32, i, m);
@@ -134,6 +138,7 @@ __global__ void __launch_bounds__(256) momentum_norm_kernel(const __grid_constan
         h[q] = pack_bf16x2(u[2 * q], u[2 * q + 1]);
         l[q] = pack_bf16x2(u[2 * q] - bf16_lo_f(h[q]), u[2 * q + 1] - bf16_hi_f(h[q]));
       }
+      if (!in_bounds(wbase + e + 8 <= nwork, p.status)) continue;
       *reinterpret_cast<uint4*>(hi + e) = make_uint4(h[0], h[1], h[2], h[3]);
       *reinterpret_cast<uint4*>(lo + e) = make_uint4(l[0], l[1], l[2], l[3]);
     }
@@ -141,9 +146,9 @@ __global__ void __launch_bounds__(256) momentum_norm_kernel(const __grid_constan
     for (long long e = e0 + threadIdx.x; e < e1; e += 256) {
       const int prow = static_cast<int>(e / Cp);
       const int pcol = static_cast<int>(e - static_cast<long long>(prow) * Cp);
+      const long long i = ubase + static_cast<long long>(prow) * C + pcol;
       float u = 0.0f;
-      if (prow < R && pcol < C) {
-        const long long i = ubase + static_cast<long long>(prow) * C + pcol;
+      if (prow < R && pcol < C && in_bounds(i < nlog, p.status)) {
         const float g = load1(io.grad, io.grad_dtype, i);
         float m = 0.0f, ms = 0.0f;
         if (p.mode != kMomNone) m = io.mom[i];
@@ -153,6 +158,7 @@ __global__ void __launch_bounds__(256) momentum_norm_kernel(const __grid_constan
         if (p.mode != kMomNone) io.mom[i] = m;
         if (p.mode == kMomAnvil) io.mom_slow[i] = ms;
       }
+      if (!in_bounds(wbase + e < nwork, p.status)) continue;
       const __nv_bfloat16 h = __float2bfloat16_rn(u);
       hi[e] = h;
       lo[e] = __float2bfloat16_rn(u - __bfloat162float(h));
@@ -213,12 +219,16 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
   const __nv_bfloat16* lo = bp.lo + mat * padded;
   const long long ubase = static_cast<long long>(mat) * bp.R * bp.C;
   const int R = bp.R, C = bp.C, Cp = bp.Cp;
+  const long long nlog = static_cast<long long>(bp.count) * R * C;  // debug-build extents
+  const long long nwork = static_cast<long long>(bp.count) * padded;
+  const long long wbase = static_cast<long long>(mat) * padded;
   if ((C & 7) == 0) {
     for (long long e = e0 + threadIdx.x * 8; e < e1; e += 256 * 8) {
       const int prow = static_cast<int>(e / Cp);
       const int pcol = static_cast<int>(e - static_cast<long long>(prow) * Cp);
       if (prow >= R || pcol >= C) continue;
       const long long i = ubase + static_cast<long long>(prow) * C + pcol;
+      if (!in_bounds(i + 8 <= nlog && wbase + e + 8 <= nwork, p.status)) continue;
       float o[8], th[8], ms[8];
       load8(hi, MUON_BF16, e, o);
       if (p.use_lo) {
@@ -251,6 +261,7 @@ __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ Upd
       const int pcol = static_cast<int>(e - static_cast<long long>(prow) * Cp);
       if (prow >= R || pcol >= C) continue;
       const long long i = ubase + static_cast<long long>(prow) * C + pcol;
+      if (!in_bounds(i < nlog && wbase + e < nwork, p.status)) continue;
       const float o = __bfloat162float(hi[e]) + (p.use_lo ? __bfloat162float(lo[e]) : 0.0f);
       if (Mode == kUpdWriteO) {
         round_store1(io.param, io.param_dtype, i, o);

@@ -279,10 +279,18 @@ __device__ __forceinline__ void epi_issue_load(const NsGemmParams& p, const EpiR
   uint64_t* bar = &e.bar[k % kEpiBufs];
   if (T.phase == kApply) {
     const int y = T.mat * bp.Rp + r0;
+    if (!in_bounds(T.mat < bp.count && r0 + kEpiRows <= bp.Rp && c0 + kEpiCols <= bp.Cp, p.status)) {
+      mbar_arrive_expect_tx(bar, 0);  // debug build: no copy, the wait still completes
+      return;
+    }
     mbar_arrive_expect_tx(bar, kEpiChunkBytes);
     tma_load_2d(b, &p.maps[T.bank][kHiE0 + T.cur], bar, c0, y);
     tma_load_2d(b + kEpiHalfBytes, &p.maps[T.bank][kLoE], bar, c0, y);
   } else if (T.phase == kPoly) {
+    if (!in_bounds(T.mat < bp.count && r0 + kEpiRows <= bp.rp && c0 + kEpiCols <= bp.rp, p.status)) {
+      mbar_arrive_expect_tx(bar, 0);
+      return;
+    }
     mbar_arrive_expect_tx(bar, kEpiHalfBytes);
     tma_load_2d(b, &p.maps[T.bank][kAE], bar, c0, T.mat * bp.rp + r0);
   }
@@ -366,6 +374,11 @@ __device__ __forceinline__ void epi_store(const NsGemmParams& p, const Tile& T, 
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
+    const int rows = T.phase == kApply ? bp.Rp : bp.rp, cols = T.phase == kApply ? bp.Cp : bp.rp;
+    if (!in_bounds(T.mat < bp.count && r0 + kEpiRows <= rows && c0 + kEpiCols <= cols, p.status)) {
+      bulk_commit();  // debug build: the chunk is not stored (an empty bulk group)
+      return;
+    }
     if (T.phase == kApply) {
       const int y = T.mat * bp.Rp + r0;
       tma_store_2d(&p.maps[T.bank][kHiE0 + (T.cur ^ 1)], buf, c0, y);

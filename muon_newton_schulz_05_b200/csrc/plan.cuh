@@ -14,6 +14,7 @@
 #include <stdint.h>
 
 #include "muon_b200.h"
+#include "check.cuh"
 #include "update_math.cuh"
 
 namespace muon {
@@ -131,6 +132,7 @@ struct MomParams {
   int sgd;            // Muon SGD-form momentum (M <- mu M + G)
   float eps;
   int mat_begin[MUON_MAX_BANKS + 1];
+  int* status;        // device status word (bounds checks of the debug build)
 };
 
 // --------------------------------------------------------------- update pass
@@ -145,6 +147,7 @@ struct UpdParams {
   int use_lo;           // O = hi + lo (else the bf16 hi alone)
   float lr_wd;          // lr * weight_decay
   float ema_beta;
+  int* status;          // device status word (bounds checks of the debug build)
 };
 
 // Launchers (defined in the .cu files).

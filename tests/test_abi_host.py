@@ -195,3 +195,24 @@ def test_other_entry_points_validate():
     assert lib.muon_device_status(None, 4096, None, 0) == 1
     assert lib.muon_set_debug(3, 1.0) == 5
     assert lib.muon_set_debug(0, 0.0) == 0
+
+
+@pytest.mark.slow
+def test_debug_build_with_bounds_checks_compiles_and_exports():
+    """`build.py --check` (-DMUON_CHECK) builds a library with every entry point
+    and the extra status code (compiled here; no GPU needed)."""
+    import importlib.util
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location(
+        "_muon_b200_build", os.path.join(root, "muon_newton_schulz_05_b200", "build.py"))
+    bld = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bld)
+    path = bld.build(check=True)
+    assert path.endswith("libmuonb200_check.so") and os.path.exists(path)
+    lib = ctypes.CDLL(path)
+    for name in mb.EXPORTED:
+        getattr(lib, name)
+    lib.muon_status_string.restype = ctypes.c_char_p
+    assert b"MUON_ERR_BOUNDS" in lib.muon_status_string(10)
+    assert mb.STATUS_NAMES[10] == "MUON_ERR_BOUNDS"
