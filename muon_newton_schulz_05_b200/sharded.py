@@ -172,6 +172,38 @@ class ShardedMuon:
             self.ema.append(state(ema))
         self._ema_ready = False
 
+    def plan_signature(self) -> Tuple:
+        """What a saved state depends on: world size, bank shapes, buckets and
+        the resulting ownership."""
+        return (self.world, tuple(self.plan.shapes),
+                tuple(tuple(bk.banks) for bk in self.plan.buckets),
+                tuple(tuple(o) for o in self.plan.owner))
+
+    def state_dict(self) -> dict:
+        """This rank's optimizer state (its owned matrices' momenta and EMA),
+        as CPU tensors, with the plan it belongs to. Save one per rank."""
+        def cpu(lists):
+            return [[t.detach().cpu().clone() if t is not None else None for t in ts] for ts in lists]
+        return {"plan": self.plan_signature(), "rank": self.rank, "variant": self.variant,
+                "momentum": cpu(self.momentum), "momentum_slow": cpu(self.momentum_slow),
+                "ema": cpu(self.ema), "ema_ready": self._ema_ready}
+
+    def load_state_dict(self, state: dict) -> None:
+        """Restore a state saved by the same rank under the same plan."""
+        if state["plan"] != self.plan_signature() or state["rank"] != self.rank:
+            raise ValueError("the state was saved under another ownership plan or rank")
+        if state["variant"] != self.variant:
+            raise ValueError("the state was saved by the other variant")
+        for name in ("momentum", "momentum_slow", "ema"):
+            mine, saved = getattr(self, name), state[name]
+            for ts, ss in zip(mine, saved):
+                for t, v in zip(ts, ss):
+                    if (t is None) != (v is None):
+                        raise ValueError(f"{name}: the saved state has a different layout")
+                    if t is not None:
+                        t.copy_(v)
+        self._ema_ready = bool(state["ema_ready"])
+
     def owned_shapes(self, k: int) -> List[Tuple[int, int, int]]:
         bk = self.plan.buckets[k]
         return [(len(o), *self.plan.shapes[b][1:]) for o, b in zip(bk.owned[self.rank], bk.banks) if o]

@@ -152,6 +152,59 @@ def test_sharded_step_equals_single_process_step(variant, buckets):
             SHAPES[b][0], -1).max(axis=1) > 0)
 
 
+def _resume_rank(rank, world, port, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from muon_newton_schulz_05_b200.sharded import ShardedMuon
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        def make():
+            return ShardedMuon(SHAPES, torch.bfloat16, torch.float32, variant="anvil",
+                               buckets=[[2], [0, 1]], ema=True,
+                               step_fn=_oracle_step_fn("anvil"), workspace_fn=lambda shapes: None)
+        hp = _hparams("anvil")
+        straight, params_a = make(), _params(SHAPES)
+        for s in range(4):
+            straight.step(params_a, _grads(SHAPES, rank, s), hp)
+        first, params_b = make(), _params(SHAPES)
+        for s in range(2):
+            first.step(params_b, _grads(SHAPES, rank, s), hp)
+        saved = first.state_dict()
+        resumed = make()              # a fresh optimizer, as after a restart
+        resumed.load_state_dict(saved)
+        for s in range(2, 4):
+            resumed.step(params_b, _grads(SHAPES, rank, s), hp)
+        same = all(torch.equal(a, b) for a, b in zip(params_a, params_b))
+        ema_a = [torch.zeros(c, r, k) for c, r, k in SHAPES]
+        ema_b = [torch.zeros(c, r, k) for c, r, k in SHAPES]
+        straight.gather_ema(ema_a)
+        resumed.gather_ema(ema_b)
+        same_ema = all(torch.equal(a, b) for a, b in zip(ema_a, ema_b))
+        wrong = ShardedMuon(SHAPES, torch.bfloat16, torch.float32, variant="anvil", ema=True,
+                            step_fn=_oracle_step_fn("anvil"), workspace_fn=lambda shapes: None)
+        try:
+            wrong.load_state_dict(saved)   # one bucket instead of two: another plan
+            rejected = False
+        except ValueError:
+            rejected = True
+        out[rank] = (same, same_ema, rejected)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_state_resumes_bitwise():
+    """2 steps, save each rank's shard state, a fresh optimizer loads it, 2
+    more steps: the same bank and EMA as 4 steps straight."""
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_resume_rank, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[0] == (True, True, True) and res[1] == (True, True, True), res
+
+
 def test_plan_owns_every_matrix_once_and_balances_gpt_bank():
     for world in (1, 2, 4, 8):
         plan = ShardPlan.build(GPT_SHAPES, world)
