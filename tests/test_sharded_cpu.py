@@ -152,6 +152,53 @@ def test_sharded_step_equals_single_process_step(variant, buckets):
             SHAPES[b][0], -1).max(axis=1) > 0)
 
 
+def _int_grads(shapes, rank, step):
+    """Integer-valued gradients: their sums over ranks are exact in any order."""
+    g = torch.Generator().manual_seed(77 * step + rank + 5)
+    return [torch.randint(-8, 9, (c, r, k), generator=g).float() for c, r, k in shapes]
+
+
+def _three_rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from muon_newton_schulz_05_b200.sharded import ShardedMuon
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        opt = ShardedMuon(SHAPES, torch.bfloat16, torch.float32, buckets=[[2], [0, 1]],
+                          step_fn=_oracle_step_fn("muon"), workspace_fn=lambda shapes: None)
+        owns = [len(o) for bk in opt.plan.buckets for o in bk.owned[rank]]
+        params = _params(SHAPES)
+        for s in range(2):
+            opt.step(params, _int_grads(SHAPES, rank, s), _hparams("muon"))
+        out[rank] = ([p.float().numpy() for p in params], owns)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_three_ranks_with_ranks_that_own_nothing_in_a_bucket():
+    """Bucket [bank 2] has one matrix: two of three ranks send and receive only
+    padding there. Every rank still ends with the single-process result."""
+    world, port = 3, _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_three_rank_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert sum(1 for r in range(world) if res[r][1][0] == 0) == 2   # bucket 0: one owner
+    from muon_newton_schulz_05_b200 import Bank
+    params = _params(SHAPES)
+    mom = [torch.zeros(c, r, k) for c, r, k in SHAPES]
+    step = _oracle_step_fn("muon")
+    for s in range(2):
+        gs = [_int_grads(SHAPES, r, s) for r in range(world)]
+        mean = [(gs[0][b] + gs[1][b] + gs[2][b]) / world for b in range(len(SHAPES))]
+        step([Bank(params[b], mean[b], mom[b]) for b in range(len(SHAPES))], _hparams("muon"), None)
+    for r in range(world):
+        for b in range(len(SHAPES)):
+            np.testing.assert_array_equal(res[r][0][b], params[b].float().numpy())
+
+
 def _resume_rank(rank, world, port, out):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
