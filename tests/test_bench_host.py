@@ -1,0 +1,35 @@
+"""Host-side pieces of the benchmark (no GPU): the flop count behind the
+roofline, the launch count and the config each JSON line carries."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import muon_inputs as mi  # noqa: E402
+import oracle  # noqa: E402
+
+
+@pytest.mark.parametrize("wid", sorted(mi.workloads()))
+def test_roofline_flops_equal_the_oracle_count(wid):
+    w = mi.workloads()[wid]
+    k = len(w.hp["coeffs"])
+    want = sum(b.count * oracle.ns_flops_algorithmic(b.rows, b.cols, k) for b in w.banks)
+    assert bench._ns_flops(w) == pytest.approx(want, rel=1e-12)
+
+
+def test_gpt_bank_chain_is_1p142_tflop():
+    # 48 x 768^2 + 24 x 768x3072 (both orientations), five steps
+    assert bench._ns_flops(mi.workloads()[bench.WORKLOAD_ID]) == pytest.approx(1.1421587866e12, rel=1e-9)
+
+
+@pytest.mark.parametrize("wid", sorted(mi.workloads()))
+def test_config_names_the_workload_and_its_cache_regime(wid):
+    w = mi.workloads()[wid]
+    c = bench._config(w)
+    assert c["workload"] and c["banks"] and c["params"] == sum(b.count * b.rows * b.cols for b in w.banks)
+    assert ("larger than L2" in c["l2"]) == (wid != 1)   # only the single 256x512 matrix fits in L2
+    assert bench.launches_per_step(w) == 4
