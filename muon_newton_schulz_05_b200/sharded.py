@@ -14,10 +14,13 @@ largest first, each to the least-loaded rank. One step, per bucket of banks:
   3. all-gather: the owners' updated parameters reach every rank, which
      unpacks them into its bank.
 
-All reduce-scatters are issued at once (asynchronous); bucket k's step waits
-only for bucket k's, so on NCCL the exchange of later buckets overlaps the
-Newton-Schulz chain of earlier ones, and each bucket's all-gather overlaps
-the next bucket's step. The packing and unpacking are plain copies; every
+`step` issues all reduce-scatters at once (asynchronous); bucket k's step
+waits only for bucket k's, so on NCCL the exchange of later buckets overlaps
+the Newton-Schulz chain of earlier ones, and each bucket's all-gather
+overlaps the next bucket's step. A training loop can start each bucket's
+exchange as soon as the backward pass has finished its gradients
+(`grad_ready(k, grads)`, every rank in the same order) and call `finish`
+after the last one. The packing and unpacking are plain copies; every
 arithmetic step of the optimizer runs in the library's kernels.
 """
 from __future__ import annotations
@@ -171,6 +174,7 @@ class ShardedMuon:
             self.momentum_slow.append(state(variant == "anvil"))
             self.ema.append(state(ema))
         self._ema_ready = False
+        self._pending: List = [None] * len(self.plan.buckets)   # reduce-scatters in flight
 
     def plan_signature(self) -> Tuple:
         """What a saved state depends on: world size, bank shapes, buckets and
@@ -209,13 +213,15 @@ class ShardedMuon:
         return [(len(o), *self.plan.shapes[b][1:]) for o, b in zip(bk.owned[self.rank], bk.banks) if o]
 
     def _reduce_scatter(self, k: int):
+        """Start bucket k's averaging reduce-scatter: its work handle, or True
+        when it is already complete (gloo)."""
         if self.gloo:
             # gloo has no reduce-scatter: sum everywhere, keep this rank's segment
             self.dist.all_reduce(self._gflat[k], op=self.dist.ReduceOp.SUM, group=self.group)
             seg = self.plan.buckets[k].seg
             self._gseg[k].copy_(self._gflat[k][self.rank * seg:(self.rank + 1) * seg])
             self._gseg[k].div_(self.world)
-            return None
+            return True
         return self.dist.reduce_scatter_tensor(self._gseg[k], self._gflat[k],
                                                op=self.dist.ReduceOp.AVG, group=self.group,
                                                async_op=True)
@@ -228,18 +234,29 @@ class ShardedMuon:
         return self.dist.all_gather_into_tensor(self._pflat[k], self._pseg[k],
                                                 group=self.group, async_op=True)
 
-    def step(self, params: Sequence, grads: Sequence, hp) -> None:
+    def grad_ready(self, k: int, grads: Sequence) -> None:
+        """Bucket k's gradients are final (grads: this rank's bank tensors, only
+        bucket k's banks are read): pack them and start their averaging
+        reduce-scatter now, so the exchange overlaps the rest of the backward
+        pass. Each bucket once per step, in any order that is the same on every
+        rank (collectives must match), then `finish`."""
+        if self._pending[k] is not None:
+            raise RuntimeError(f"bucket {k} is already in flight in this step")
+        self.plan.pack(k, grads, self._gflat[k])
+        self._pending[k] = self._reduce_scatter(k)
+
+    def finish(self, params: Sequence, hp) -> None:
+        """Step every bucket whose reduce-scatter `grad_ready` started (all must
+        have been), in bucket order, and bring the updated parameters to
+        every rank."""
         from . import Bank
         plan, rank = self.plan, self.rank
-        nb = len(plan.buckets)
-        rs = []
-        for k in range(nb):
-            plan.pack(k, grads, self._gflat[k])
-            rs.append(self._reduce_scatter(k))
+        if any(w is None for w in self._pending):
+            raise RuntimeError("every bucket needs grad_ready before finish")
         ag = []
         for k, bk in enumerate(plan.buckets):
-            if rs[k] is not None:
-                rs[k].wait()
+            if self._pending[k] is not True:
+                self._pending[k].wait()
             gv = plan.views(k, rank, self._gseg[k])
             pv = plan.views(k, rank, self._pseg[k])
             banks = []
@@ -256,11 +273,18 @@ class ShardedMuon:
                     self._init_ema(k, pv)
                 self.step_fn(banks, hp, self.workspaces[k])
             ag.append(self._all_gather(k))
-        for k in range(nb):
+        for k in range(len(plan.buckets)):
             if ag[k] is not None:
                 ag[k].wait()
             plan.unpack(k, self._pflat[k], params)
+        self._pending = [None] * len(plan.buckets)
         self._ema_ready = True
+
+    def step(self, params: Sequence, grads: Sequence, hp) -> None:
+        """One data-parallel step: every bucket's exchange, then `finish`."""
+        for k in range(len(self.plan.buckets)):
+            self.grad_ready(k, grads)
+        self.finish(params, hp)
 
     def _init_ema(self, k: int, pv) -> None:
         # the average starts at the parameters it averages

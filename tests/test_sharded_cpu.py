@@ -199,6 +199,52 @@ def test_three_ranks_with_ranks_that_own_nothing_in_a_bucket():
             np.testing.assert_array_equal(res[r][0][b], params[b].float().numpy())
 
 
+def _split_rank(rank, world, port, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from muon_newton_schulz_05_b200.sharded import ShardedMuon
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        def make():
+            return ShardedMuon(SHAPES, torch.bfloat16, torch.float32, buckets=[[0], [1], [2]],
+                               step_fn=_oracle_step_fn("muon"), workspace_fn=lambda shapes: None)
+        hp = _hparams("muon")
+        a, pa = make(), _params(SHAPES)
+        b, pb = make(), _params(SHAPES)
+        for s in range(2):
+            g = _grads(SHAPES, rank, s)
+            a.step(pa, g, hp)
+            for k in (2, 1, 0):        # the backward pass finishes the last bucket first
+                b.grad_ready(k, g)
+            b.finish(pb, hp)
+        same = all(torch.equal(x, y) for x, y in zip(pa, pb))
+        errors = []
+        try:
+            b.finish(pb, hp)            # no bucket is ready
+        except RuntimeError:
+            errors.append("finish")
+        b.grad_ready(0, _grads(SHAPES, rank, 9))
+        try:
+            b.grad_ready(0, _grads(SHAPES, rank, 9))
+        except RuntimeError:
+            errors.append("twice")
+        out[rank] = (same, errors)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_grad_ready_then_finish_equals_step():
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_split_rank, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    for r in (0, 1):
+        assert res[r] == (True, ["finish", "twice"]), res
+
+
 def _resume_rank(rank, world, port, out):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
