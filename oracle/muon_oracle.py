@@ -73,6 +73,8 @@ __all__ = [
     "muon_step",
     "anvil_step",
     "ema_update",
+    "weighted_average",
+    "weighted_average_betas",
     "readout_blend",
     "ns_flops_algorithmic",
 ]
@@ -256,6 +258,37 @@ def ema_update(ema: np.ndarray, theta: np.ndarray, beta: float) -> np.ndarray:
     """theta_bar <- beta theta_bar + (1 - beta) theta
     ([P3] "ANVIL II와 가중치 평균", the averaging equation)."""
     return beta * as_f64(ema) + (1.0 - beta) * as_f64(theta)
+
+
+def weighted_average(thetas: Sequence, weights: Sequence[float]) -> np.ndarray:
+    """theta_bar = sum_i w_i theta_i / sum_i w_i over checkpoints theta_i.
+
+    "qlabs-eng/slowrun", leaderboard table: weighted checkpoint averaging. The
+    page gives no weights, so they are the caller's (w_i >= 0, sum > 0). The
+    EMA of "ANVIL II와 가중치 평균" is the special case w_0 = beta^n,
+    w_i = (1 - beta) beta^(n - i).
+    """
+    w = [float(x) for x in weights]
+    if len(w) != len(thetas) or not w or min(w) < 0.0 or sum(w) <= 0.0:
+        raise ValueError("need one non-negative weight per checkpoint, not all zero")
+    acc = np.zeros_like(as_f64(thetas[0]))
+    for wi, th in zip(w, thetas):
+        acc = acc + wi * as_f64(th)
+    return acc / sum(w)
+
+
+def weighted_average_betas(weights: Sequence[float]) -> list:
+    """The decay of each checkpoint that makes the EMA recurrence
+    theta_bar <- beta_n theta_bar + (1 - beta_n) theta_n produce the running
+    weighted average: beta_n = 1 - w_n / W_n with W_n = w_1 + ... + w_n
+    (beta_1 = 0, so the average starts at the first checkpoint). Checkpoints
+    before the first positive weight get beta = 1 - 0 / 0, taken as 0 here
+    (they are overwritten by the first weighted one)."""
+    out, W = [], 0.0
+    for wn in weights:
+        W += float(wn)
+        out.append(1.0 - float(wn) / W if W > 0.0 else 0.0)
+    return out
 
 
 def readout_blend(theta: np.ndarray, ema: np.ndarray, w_final: float = 0.35) -> np.ndarray:

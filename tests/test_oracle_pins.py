@@ -326,3 +326,113 @@ def test_pin_catches_plausible_mistakes():
         for bad in (wrong_sign, dropped_square, gram_transposed):
             err = _closed_form_error(bad)
             assert not (err < 1e-3), bad.__name__
+
+
+# ---- ANVIL: which momentum gets which beta, and what each one feeds --------
+def test_anvil_step_wiring_three_steps_closed_form():
+    """Three anvil_step calls from non-zero momenta with beta_fast != beta_slow,
+    against closed forms written out by hand.
+
+    The gradient is the same positive rank-one matrix G = u v^T every step and
+    both momenta start as multiples of it (M_fast) or of a fixed sign pattern
+    (M_slow), so after step t
+      M_fast_t = beta_f^t M_fast_0 + (1 - beta_f^t) G          (a multiple of G)
+      M_slow_t = beta_s^t M_slow_0 + (1 - beta_s^t) G.
+    O is the Newton-Schulz image of the rank-one fast momentum: sign(k) times
+    p^6(s0) times the unit rank-one direction. The start values are chosen so
+    that the sign of k and the slow momentum's sign on part of the entries
+    both flip if the two betas are exchanged ("ANVIL II와 가중치 평균": the fast
+    momentum is the update, the slow one only picks where the decay applies).
+    """
+    rows, cols = 4, 6
+    u = np.linspace(1.0, 2.0, rows)
+    v = np.linspace(0.5, 1.5, cols)
+    G = np.outer(u, v)                      # entries in [0.5, 3]
+    bf, bs = 0.9, 0.99
+    k0 = -0.08                              # M_fast_0 = k0 G
+    pattern = np.where(np.arange(rows * cols).reshape(rows, cols) % 2 == 0, -0.5, 0.5)
+    th = np.full((rows, cols), 0.25)
+    lr, wd, eps = 0.05, 0.4, 1e-7
+    coeffs = [QUINTIC] * 6
+    hp = dict(lr=lr, beta_fast=bf, beta_slow=bs, weight_decay=wd, coeffs=coeffs, eps=eps)
+    Mf, Ms = k0 * G, pattern.copy()
+    unit = np.outer(u / np.linalg.norm(u), v / np.linalg.norm(v))
+    gnorm = np.linalg.norm(u) * np.linalg.norm(v)
+    flipped = 0
+    for t in (1, 2, 3):
+        th_new, Mf, Ms, O, mask = oracle.anvil_step(th, G, Mf, Ms, hp, "f32")
+        k = bf ** t * k0 + (1 - bf ** t)
+        assert np.max(np.abs(Mf - k * G)) < 1e-14
+        Ms_exp = bs ** t * pattern + (1 - bs ** t) * G
+        assert np.max(np.abs(Ms - Ms_exp)) < 1e-14
+        s0 = abs(k) * gnorm / (abs(k) * gnorm + eps)
+        O_exp = np.sign(k) * _scalar_orbit([s0], coeffs)[0] * unit
+        assert np.max(np.abs(O - O_exp)) < 1e-12
+        mask_exp = (O_exp * Ms_exp > 0).astype(float)
+        assert np.array_equal(mask, mask_exp)
+        th_exp = th - lr * wd * mask_exp * th - lr * 1.0 * O_exp
+        assert np.max(np.abs(th_new - th_exp.astype(np.float32))) <= 1e-7
+        # with the betas exchanged the fast coefficient changes sign and the
+        # slow momentum changes sign on some entries
+        k_sw = bs ** t * k0 + (1 - bs ** t)
+        Ms_sw = bf ** t * pattern + (1 - bf ** t) * G
+        assert np.sign(k_sw) != np.sign(k)
+        flipped += int(np.sum(np.sign(Ms_sw) != np.sign(Ms_exp)))
+        th = th_new
+    assert flipped > 0
+
+
+# ---- weighted checkpoint average ------------------------------------------
+def test_weighted_average_three_checkpoints_by_hand():
+    """theta_1 = (1, 2), theta_2 = (3, -1), theta_3 = (0, 4), w = (1, 2, 5):
+    (1*(1,2) + 2*(3,-1) + 5*(0,4)) / 8 = (7/8, 20/8)."""
+    thetas = [np.array([1.0, 2.0]), np.array([3.0, -1.0]), np.array([0.0, 4.0])]
+    got = oracle.weighted_average(thetas, [1.0, 2.0, 5.0])
+    assert np.array_equal(got, np.array([0.875, 2.5]))
+    # the running form: beta = (0, 1 - 2/3, 1 - 5/8)
+    betas = oracle.weighted_average_betas([1.0, 2.0, 5.0])
+    assert betas[0] == 0.0 and abs(betas[1] - 1.0 / 3.0) < 1e-16 and betas[2] == 0.375
+    e = thetas[0]
+    for b, th in zip(betas, thetas):
+        e = oracle.ema_update(e, th, b)
+    assert np.max(np.abs(e - np.array([0.875, 2.5]))) < 1e-15
+
+
+def test_weighted_average_running_form_exact_rationals():
+    """The beta schedule reproduces the weighted average exactly (Fraction)."""
+    rng = np.random.default_rng(4)
+    ths = [[Fraction(int(x), 7) for x in rng.integers(-20, 20, 3)] for _ in range(6)]
+    ws = [Fraction(int(x), 3) for x in rng.integers(1, 9, 6)]
+    W = sum(ws)
+    exact = [sum(w * t[j] for w, t in zip(ws, ths)) / W for j in range(3)]
+    e = list(ths[0])
+    Wn = Fraction(0)
+    for w, t in zip(ws, ths):
+        Wn += w
+        beta = 1 - w / Wn
+        e = [beta * a + (1 - beta) * b for a, b in zip(e, t)]
+    assert e == exact
+    got = oracle.weighted_average([np.array([float(x) for x in t]) for t in ths],
+                                  [float(w) for w in ws])
+    assert np.allclose(got, [float(x) for x in exact], rtol=1e-14, atol=1e-15)
+    betas = oracle.weighted_average_betas([float(w) for w in ws])
+    e = np.array([float(x) for x in ths[0]])
+    for b, t in zip(betas, ths):
+        e = oracle.ema_update(e, np.array([float(x) for x in t]), b)
+    assert np.allclose(e, [float(x) for x in exact], rtol=1e-13, atol=1e-14)
+
+
+def test_ema_is_a_weighted_average():
+    """The EMA from theta_bar_0 = theta_0 equals the weighted average with
+    w_0 = beta^n and w_i = (1 - beta) beta^(n - i)."""
+    rng = np.random.default_rng(8)
+    ths = [rng.standard_normal((3, 4)) for _ in range(5)]
+    beta = 0.9
+    e = ths[0].copy()
+    for th in ths[1:]:
+        e = oracle.ema_update(e, th, beta)
+    n = len(ths) - 1
+    w = [beta ** n] + [(1 - beta) * beta ** (n - i) for i in range(1, n + 1)]
+    assert np.max(np.abs(oracle.weighted_average(ths, w) - e)) < 1e-14
+    with pytest.raises(ValueError):
+        oracle.weighted_average(ths, [0.0] * len(ths))
