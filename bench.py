@@ -5,14 +5,14 @@ Workload: 48 x 768x768, 12 x 768x3072, 12 x 3072x768 bf16 parameters (84.9 M),
 bf16 gradients N(0, 1e-3^2) plus a rank-4 spike at 10x RMS, fp32 momentum,
 mu = 0.95 Nesterov, five quintic Newton-Schulz steps (3.4445, -4.7750, 2.0315),
 lr 0.05, no weight decay. A step is one muon_step over the whole bank:
-momentum + norm -> 15 Newton-Schulz GEMM launches -> scaled parameter write.
+momentum + norm -> the Newton-Schulz chain (one persistent launch: every
+step, phase and matrix) -> scaled parameter write.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-N > 1 runs under torchrun, one process per GPU; every rank steps its own
-bank (independent problems, no collective on the data path: weak scaling) and
-rank 0 prints one JSON line with the max-over-ranks device time.
-`--impl reference` times the CPU oracle (host cores) on a bounded sample.
+The same run also times the 64 x 1024^2 bank (20 steps after 3 warm-up
+steps) for its Newton-Schulz roofline line.
+`--impl reference` times the CPU oracle (host cores) on the whole bank.
 """
 from __future__ import annotations
 
@@ -31,10 +31,14 @@ sys.path.insert(0, ROOT)
 METRIC = "Muon steps/s on GPT-124M matrix bank; NS TFLOP/s as % bf16 tensor peak"
 UNIT = "steps/s"
 WORKLOAD_ID = 2
-# DRAM bytes (read + write) of one Newton-Schulz chain launch on this workload,
-# from the ncu capture summarised in profiles/ns_gemm_gpt124m_bank.md. Set to
-# None whenever ns_gemm_kernel changes until it is captured again.
-NS_CHAIN_DRAM_BYTES = 5.191235e9
+SQUARE_ID = 3
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# Newton-Schulz chain launch per workload, from an ncu capture of one chain
+# launch, with a hash of the kernel sources it was taken from: once the
+# sources change the figure no longer describes the kernel and is reported
+# as null.
+NS_CHAIN_TRAFFIC = {}
+KERNEL_SOURCES = ("ns_gemm.cu", "plan.cuh", "ptx.cuh")
 
 
 def launches_per_step(w) -> int:
@@ -51,6 +55,8 @@ def _args():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-square", action="store_true",
+                    help="skip the 64 x 1024^2 roofline line")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
                     help="1..5 (default 2, the GPT-124M bank the metric names); the others "
                          "are measured for documentation only")
@@ -65,6 +71,26 @@ def _peaks():
                     sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]), src="measured")
     except Exception:
         return dict(hbm=6650.0, burst=1590.0, sustained=1400.0, src="fallback")
+
+
+def kernel_source_sha16() -> str:
+    """Hash of the Newton-Schulz kernel's sources (what a traffic figure describes)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "muon_newton_schulz_05_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def chain_traffic(wid: int):
+    """(bytes per chain launch, where from) or (None, why not)."""
+    t = NS_CHAIN_TRAFFIC.get(wid)
+    if t is None:
+        return None, "no ncu capture of this workload's chain launch"
+    if t["source_sha16"] != kernel_source_sha16():
+        return None, "the kernel sources changed since the ncu capture"
+    return t["bytes"], t["capture"]
 
 
 def _workload(wid: int = WORKLOAD_ID):
@@ -137,37 +163,55 @@ def _cpu_threads():
     return len(os.sched_getaffinity(0))
 
 
-def _oracle_sample_time(w, budget_s: float, start_step: int = 0, max_per_shape: int = 12):
-    """Oracle Muon step on matrices of the bank, cycling the three shapes,
-    until budget_s of CPU work; returns (seconds per full-bank step, sample
-    description)."""
+_PARAM_CACHE = {}
+
+
+def _oracle_bank_time(w, step: int = 0, max_layers=None):
+    """Seconds of one oracle step over the whole bank (every matrix, one after
+    another, float64), and a description. The gradients are generated and
+    converted outside the timed calls. For a bank too large to time in full
+    (max_layers set), the first max_layers matrices of each shape are timed
+    and the time is scaled by the bank's counts, labelled as extrapolated."""
     import numpy as np
     import muon_inputs as mi
     import oracle
-    per_shape = {b: [] for b in range(len(w.banks))}
-    t_start = time.perf_counter()
-    idx = 0
-    while True:
-        for b, spec in enumerate(w.banks):
-            i = idx % spec.count
-            th = oracle.as_f64(mi.make_params(w, b, [i])[0])
-            g = oracle.as_f64(mi.make_grads(w, b, start_step, [i])[0])
+    total, n, scaled = 0.0, 0, False
+    for b, spec in enumerate(w.banks):
+        count = spec.count if max_layers is None else min(spec.count, max_layers)
+        key = (w.cid, b, count)
+        if key not in _PARAM_CACHE:  # the parameters are the same every step
+            _PARAM_CACHE[key] = mi.make_params(w, b, list(range(count)))
+        t_bank = 0.0
+        for i in range(count):
+            th = oracle.as_f64(_PARAM_CACHE[key][i])
+            g = oracle.as_f64(mi.make_grads(w, b, step, [i])[0])
             m = np.zeros_like(g)
             t0 = time.perf_counter()
             if w.variant == "anvil":
                 oracle.anvil_step(th, g, m, m, w.hp, w.param_dtype)
             else:
                 oracle.muon_step(th, g, m, w.hp, w.param_dtype)
-            per_shape[b].append(time.perf_counter() - t0)
-        idx += 1
-        if time.perf_counter() - t_start >= budget_s or idx >= max(1, min(12, max_per_shape)):
-            break
-    full = sum(w.banks[b].count * statistics.mean(ts) for b, ts in per_shape.items())
-    n = sum(len(ts) for ts in per_shape.values())
-    desc = (f"oracle {w.variant}_step (float64, numpy) on {n} matrices ({idx} of each shape "
-            f"{', '.join(f'{s.rows}x{s.cols}' for s in w.banks)}), mean time per shape "
-            f"scaled by the bank's counts {[s.count for s in w.banks]}")
-    return full, desc
+            t_bank += time.perf_counter() - t0
+            n += 1
+        if count < spec.count:
+            scaled = True
+            t_bank *= spec.count / count
+        total += t_bank
+    shapes = ", ".join(f"{s.count}x{s.rows}x{s.cols}" for s in w.banks)
+    if scaled:
+        desc = (f"oracle {w.variant}_step (float64, numpy) on the first {max_layers} matrices of "
+                f"each shape of the bank {shapes} ({n} matrices), scaled by the bank's counts "
+                f"(extrapolated)")
+    else:
+        desc = (f"oracle {w.variant}_step (float64, numpy) on every matrix of the bank "
+                f"{shapes} ({n} matrices), one full step")
+    return total, desc
+
+
+def _oracle_layers(w):
+    """Whole bank, except the 2.5B bank (about 161 dense TFLOP per step in
+    float64): one matrix of each shape, extrapolated."""
+    return 1 if w.n_params > 1_000_000_000 else None
 
 
 def run_reference(args):
@@ -175,14 +219,15 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = _workload(args.workload)
-    for _ in range(args.warmup):
-        _oracle_sample_time(w, 0.0)
+    layers = _oracle_layers(w)
+    for s in range(args.warmup):
+        _oracle_bank_time(w, s, layers)
     times = []
     desc = ""
     for s in range(args.steps):
-        t, desc = _oracle_sample_time(w, 0.0, start_step=s)
+        t, desc = _oracle_bank_time(w, args.warmup + s, layers)
         times.append(t)
-    spb = statistics.median(times)
+    spb = sum(times) / len(times)
     v = 1.0 / spb
     cores = _cpu_threads()
     line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
@@ -190,7 +235,7 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference", "config": _config(w),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": "each step: " + desc},
+                             "sample": f"each of the {args.steps} timed steps: " + desc},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -393,9 +438,13 @@ def run_native(args):
                        "through the public API, device->host copy of the updated parameters; "
                        "copies of neighbouring steps overlap the step on two copy streams"}
 
+    square = None
+    if args.workload == WORKLOAD_ID and not args.no_square:
+        square = _square_roofline(args, dev, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        spb, desc = _oracle_sample_time(w, 15.0)
+        spb, desc = _oracle_bank_time(w, 0, _oracle_layers(w))
         cpu = {"value": 1.0 / spb, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
                "sample": desc}
 
@@ -404,24 +453,14 @@ def run_native(args):
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    peak = peaks["sustained"]
+    traffic, traffic_src = chain_traffic(args.workload)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": _config(w),
-        "roofline": {
-            "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak,
-            "traffic": NS_CHAIN_DRAM_BYTES if args.workload == WORKLOAD_ID else None,
-            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
-                              "(profiles/ns_gemm_gpt124m_bank.md)",
-            "kernel": "ns_gemm_kernel (one persistent launch: every Newton-Schulz step x "
-                      "Gram/Poly/Apply over the bank)",
-            "flops_per_launch": flops_step, "launch_ms": ns_avg_ms,
-            "peak_kind": f"bf16 dense sustained, {peaks['src']}",
-            "frac_of_burst": achieved / peaks["burst"],
-        },
+        "roofline": _roofline(achieved, peaks, flops_step, ns_avg_ms, traffic, traffic_src),
+        "roofline_square_1024x1024x64": square,
         "breakdown_ms": {"momentum_norm": statistics.mean(pre_ms), "ns_chain": ns_avg_ms,
                          "update": statistics.mean(post_ms)},
         "elementwise_gbs": {"momentum_norm": pre_gbs, "update": post_gbs, "peak": peaks["hbm"]},
@@ -430,6 +469,56 @@ def run_native(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _roofline(achieved, peaks, flops, launch_ms, traffic, traffic_src):
+    """The chain's roofline object. The timed region is well under a second,
+    so the denominator is the measured burst bf16 peak; the fraction of the
+    sustained (power-capped) peak is reported beside it."""
+    return {
+        "bound": "tensor", "achieved": achieved, "peak": peaks["burst"], "unit": "TFLOP/s",
+        "frac": achieved / peaks["burst"], "traffic": traffic, "traffic_source": traffic_src,
+        "kernel": "ns_gemm_kernel (one persistent launch: every Newton-Schulz step x "
+                  "Gram/Poly/Apply over the bank)",
+        "flops_per_launch": flops, "launch_ms": launch_ms,
+        "peak_kind": f"bf16 dense burst, {peaks['src']} (timed region under a second)",
+        "frac_of_sustained": achieved / peaks["sustained"],
+    }
+
+
+def _square_roofline(args, dev, peaks, steps=20, warmup=3):
+    """Newton-Schulz roofline on the 64 x 1024^2 bank (inputs resident, 20
+    timed steps after 3 warm-up steps; chain bracketed with CUDA events)."""
+    import torch
+    import muon_inputs as mi
+    import muon_newton_schulz_05_b200 as mb
+    w = _workload(SQUARE_ID)
+    banks = []
+    for b in range(len(w.banks)):
+        th = mi.make_params(w, b).to(dev)
+        banks.append(mb.Bank(th, mi.make_grads(w, b, 0).to(dev),
+                             torch.zeros(th.shape, dtype=torch.float32, device=dev)))
+    ws = mb.alloc_workspace([bk.shape for bk in banks], device=dev)
+    H = mb.Hparams.from_dict(w.hp)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        mb.muon_step(banks, H, ws)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+    torch.cuda.synchronize()
+    for s_ in range(steps):
+        mb.set_ns_events(ev[2 * s_], ev[2 * s_ + 1])
+        mb.muon_step(banks, H, ws)
+    torch.cuda.synchronize()
+    assert mb.device_status(ws) == 0
+    ns_ms = statistics.mean(ev[2 * s_].elapsed_time(ev[2 * s_ + 1]) for s_ in range(steps))
+    flops = _ns_flops(w)
+    traffic, src = chain_traffic(SQUARE_ID)
+    r = _roofline(flops / (ns_ms * 1e-3) / 1e12, peaks, flops, ns_ms, traffic, src)
+    r["workload"] = "64 x 1024x1024 bf16, quintic x5, mu 0.95, wd 0.01 (inputs resident)"
+    r["steps"], r["warmup"] = steps, warmup
+    del banks, ws
+    torch.cuda.empty_cache()
+    return r
 
 
 def main():

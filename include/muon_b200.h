@@ -31,8 +31,21 @@
  *     allocates, frees or synchronises in the step calls; work is enqueued on
  *     `stream` (a cudaStream_t passed as void*, NULL = legacy default stream).
  *   - Arguments are validated on the host before anything is enqueued; a
- *     non-OK status means nothing was launched. Faults found on the device
- *     (a bounded wait that ran out) are reported by muon_device_status.
+ *     non-OK status means nothing was launched. MUON_OK from a step call
+ *     means only that its work was enqueued. Faults found on the device (a
+ *     bounded wait that ran out) are recorded in the workspace's status word
+ *     and reported by muon_device_status, which synchronises: call it
+ *     outside the hot loop, e.g. once every N steps or at a checkpoint.
+ *   - The status word is sticky. In the step whose chain timed out the
+ *     momenta have already advanced (the momentum pass runs first), but
+ *     param, ema and O are left unchanged; every later step on that
+ *     workspace leaves all of its buffers unchanged until the word is
+ *     cleared (muon_device_status with clear != 0). Restore the momenta from
+ *     a checkpoint before resuming if the failed step must not count.
+ *   - One Newton-Schulz chain is a persistent launch whose CTA pairs wait on
+ *     one another; its grid is capped at the pairs the device can hold at
+ *     once. Chains on several streams of one device are correct but
+ *     serialise; kernels of other streams that hold SMs delay a chain.
  *   - Every device pointer must be 16-byte aligned. param, momentum,
  *     momentum_slow and ema are updated in place and must not overlap one
  *     another, in the same bank or in another bank of the call (checked:

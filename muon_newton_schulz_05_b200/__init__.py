@@ -144,9 +144,7 @@ class Hparams:
         h = CHparams()
         h.lr, h.mu, h.weight_decay, h.eps = self.lr, self.mu, self.weight_decay, self.eps
         h.nesterov = 1 if self.nesterov else 0
-        h.ns_steps = len(self.coeffs)
-        if not 1 <= h.ns_steps <= MAX_NS_STEPS:
-            h.ns_steps = len(self.coeffs)  # validated by the library
+        h.ns_steps = len(self.coeffs)  # range checked by the library (MUON_ERR_HPARAM)
         for i, (a, b, c) in enumerate(list(self.coeffs)[:MAX_NS_STEPS]):
             h.coeffs[3 * i], h.coeffs[3 * i + 1], h.coeffs[3 * i + 2] = a, b, c
         h.ema_beta, h.beta_fast, h.beta_slow = self.ema_beta, self.beta_fast, self.beta_slow
@@ -247,6 +245,25 @@ def ema_update(banks: Sequence[Bank], beta: float, stream=None) -> None:
     _check(_lib.ema_update(arr, len(banks), beta, _stream_handle(stream)), "ema_update")
 
 
+def checkpoint_average_betas(weights: Sequence[float]) -> List[float]:
+    """The beta of each ema_update call that turns the EMA recurrence into a
+    weighted checkpoint average sum_i w_i theta_i / sum_i w_i: checkpoint n
+    uses beta_n = 1 - w_n / (w_1 + ... + w_n) (so beta_1 = 0: the average
+    starts at the first checkpoint). A checkpoint with weight 0 gets beta = 1,
+    which ema_update rejects: skip its call instead. Host scalars only; the
+    averaging itself is ema_update's kernel."""
+    out, total = [], 0.0
+    for w in weights:
+        w = float(w)
+        if w < 0.0:
+            raise ValueError("checkpoint weights must be non-negative")
+        total += w
+        if total <= 0.0:
+            raise ValueError("the first checkpoint needs a positive weight")
+        out.append(1.0 - w / total)
+    return out
+
+
 def readout_blend(theta, ema, out, w_final: float = 0.35, stream=None) -> None:
     _check(_lib.readout_blend(_ptr(theta), _dtype_code(theta), _ptr(ema), _ptr(out),
                               _dtype_code(out), theta.numel(), w_final, _stream_handle(stream)),
@@ -282,5 +299,6 @@ def loaded_library_path() -> str:
 
 __all__: List[str] = ["Bank", "Hparams", "MuonError", "workspace_size", "alloc_workspace",
                       "muon_step", "anvil_step", "orthogonalize", "ema_update", "readout_blend",
+                      "checkpoint_average_betas",
                       "device_status", "set_debug", "set_ns_events", "status_string", "abi_version",
                       "raw_library", "CBank", "CHparams", "EXPORTED", "F32", "BF16"]

@@ -30,10 +30,11 @@ std::mutex g_mu;
 struct DeviceState {
   bool ready = false;
   int sms = 0;
+  int max_pairs = 0;  // CTA pairs of the Newton-Schulz chain that fit on the device at once
 };
 DeviceState g_dev[64];
 
-muon_status device_state(int* sms) {
+muon_status device_state(int* sms, int* max_pairs = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MUON_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -50,10 +51,11 @@ muon_status device_state(int* sms) {
   if (!d.ready) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return MUON_ERR_CUDA;
-    if (ns_gemm_prepare() != cudaSuccess) return MUON_ERR_CUDA;
+    if (ns_gemm_prepare(&d.max_pairs) != cudaSuccess) return MUON_ERR_CUDA;
     d.ready = true;
   }
   *sms = d.sms;
+  if (max_pairs) *max_pairs = d.max_pairs;
   return MUON_OK;
 }
 
@@ -262,8 +264,8 @@ UpdBank update_io(const muon_bank& b, const muon_hparams* hp) {
 
 muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_hparams* hp,
                      void* ws, size_t ws_bytes, cudaStream_t stream, const OrthoIO* oio) {
-  int sms = 0;
-  muon_status st = device_state(&sms);
+  int sms = 0, max_pairs = 0;
+  muon_status st = device_state(&sms, &max_pairs);
   if (st != MUON_OK) return st;
 
   Shape3 shapes[MUON_MAX_BANKS];
@@ -274,6 +276,10 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   const size_t need = plan_workspace(shapes, nbanks, static_cast<uint8_t*>(ws), plans);
   if (ws_bytes < need) return MUON_ERR_WORKSPACE;
   int* status = static_cast<int*>(ws);
+  // every fallible host-side step comes before the first launch, so an error
+  // return means that nothing was enqueued (the momenta are not advanced)
+  for (int b = 0; b < nbanks; ++b)
+    if ((st = encode_bank_maps(plans[b], gp.maps[b])) != MUON_OK) return st;
 
   // ---- momentum + norm partials, then 1/(||U||+eps)
   MomParams mp;
@@ -309,10 +315,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   const double lim = g_debug.wait_limit_s > 0 ? g_debug.wait_limit_s : 2.0;
   gp.wait_limit_ns = static_cast<unsigned long long>(lim * 1e9);
   gp.fault = g_debug.fault;
-  for (int b = 0; b < nbanks; ++b) {
-    gp.bank[b] = plans[b];
-    if ((st = encode_bank_maps(plans[b], gp.maps[b])) != MUON_OK) return st;
-  }
+  for (int b = 0; b < nbanks; ++b) gp.bank[b] = plans[b];
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -338,7 +341,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   gp.red_begin[nbanks] = red;
   gp.sym_begin[nbanks] = sym;
   gp.apply_begin[nbanks] = app;
-  if (launch_ns_gemm(gp, sms, stream) != cudaSuccess) return MUON_ERR_CUDA;
+  if (launch_ns_gemm(gp, max_pairs, stream) != cudaSuccess) return MUON_ERR_CUDA;
   if (ev_after && cudaEventRecord(ev_after, stream) != cudaSuccess) return MUON_ERR_CUDA;
 
   // ---- scale, decay, parameter write (+ EMA), or O out

@@ -88,8 +88,18 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
   return t;
 }
 
+// Every pass that writes the caller's buffers first reads the workspace's
+// status word: while it holds an error (a bounded wait of an earlier launch
+// ran out; the word is sticky until the caller clears it) the pass writes
+// nothing, so a failed step leaves params, EMA and O as they were, and later
+// steps leave the momenta too.
+__device__ __forceinline__ bool status_clear(const int* status) {
+  return status == nullptr || *reinterpret_cast<const volatile int*>(status) == 0;
+}
+
 __global__ void __launch_bounds__(256) momentum_norm_kernel(const __grid_constant__ MomParams p) {
   __shared__ float red[8];
+  if (!status_clear(p.status)) return;
   const int blk = blockIdx.x;
   int b = 0;
   while (b + 1 < p.nbanks && blk >= p.block_begin[b + 1]) ++b;
@@ -204,6 +214,7 @@ cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total
 // version with two groups per thread reached about half of the bandwidth).
 template <int Mode>
 __global__ void __launch_bounds__(256) update_kernel(const __grid_constant__ UpdParams p) {
+  if (!status_clear(p.status)) return;  // the chain did not finish: O is not valid
   const int blk = blockIdx.x;
   int b = 0;
   while (b + 1 < p.nbanks && blk >= p.block_begin[b + 1]) ++b;

@@ -208,7 +208,12 @@ __device__ __forceinline__ bool wait_dependency(const int* cnt, int target, vola
       __nanosleep(64);
       if (ld_acquire_gpu(cnt) >= target) break;
       if ((i & 15u) == 0) {
-        if (*abort) return false;
+        // another CTA's wait ran out (or an earlier launch's): the counter may
+        // never reach the target, so give up at once
+        if (*abort || *reinterpret_cast<volatile int*>(status)) {
+          *abort = 1;
+          return false;
+        }
         if (global_timer_ns() - t0 > limit_ns) {
           *abort = 1;
           atomicExch(status, 8 /* MUON_ERR_TIMEOUT */);
@@ -760,14 +765,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-cudaError_t ns_gemm_prepare() {
-  return cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              kGemmSmemBytes);
+// One-time set-up on the current device: the kernel's shared-memory size and
+// the number of CTA pairs that can be resident at once. The chain's tiles
+// wait on tiles that other pairs own, so every pair of the grid must be
+// resident together; the grid never exceeds what the occupancy calculator
+// reports for this kernel's cluster and shared-memory configuration (on an
+// otherwise idle device: one pair per TPC). Kernels of other streams that hold
+// SMs only delay the pairs that cannot start yet; chains on several streams
+// of one device serialise the same way.
+cudaError_t ns_gemm_prepare(int* max_pairs) {
+  cudaError_t e = cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kGemmSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters, ns_gemm_kernel, &cfg)) != cudaSuccess) return e;
+  if (clusters < 1) return cudaErrorInvalidConfiguration;
+  *max_pairs = clusters < sms / 2 ? clusters : sms / 2;
+  return cudaSuccess;
 }
 
-cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s) {
+cudaError_t launch_ns_gemm(const NsGemmParams& p, int max_pairs, cudaStream_t s) {
   const int tiles = p.ns_steps * tiles_per_step(p);
-  int pairs = num_sms / 2;
+  int pairs = max_pairs;
   if (tiles < pairs) pairs = tiles;
   if (pairs < 1) pairs = 1;
   ns_gemm_kernel<<<2 * pairs, kGemmThreads, kGemmSmemBytes, s>>>(p);

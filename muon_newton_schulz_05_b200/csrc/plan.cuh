@@ -153,12 +153,12 @@ struct UpdParams {
 // Launchers (defined in the .cu files).
 cudaError_t launch_momentum_norm(const MomParams& p, int total_blocks, int total_mats,
                                  cudaStream_t s);
-cudaError_t launch_ns_gemm(const NsGemmParams& p, int num_sms, cudaStream_t s);  // whole chain
+cudaError_t launch_ns_gemm(const NsGemmParams& p, int max_pairs, cudaStream_t s);  // whole chain
 cudaError_t launch_update(const UpdParams& p, int total_blocks, cudaStream_t s);
 cudaError_t launch_ema(float* ema, const void* param, int param_dtype, long long n, float beta,
                        int num_sms, cudaStream_t s);
 cudaError_t launch_blend(const void* theta, int theta_dtype, const float* ema, void* out,
                          int out_dtype, long long n, float w_final, int num_sms, cudaStream_t s);
-cudaError_t ns_gemm_prepare();   // one-time function attributes
+cudaError_t ns_gemm_prepare(int* max_pairs);  // one-time attributes; co-resident CTA pairs
 
 }  // namespace muon

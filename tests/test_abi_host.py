@@ -216,3 +216,15 @@ def test_debug_build_with_bounds_checks_compiles_and_exports():
     lib.muon_status_string.restype = ctypes.c_char_p
     assert b"MUON_ERR_BOUNDS" in lib.muon_status_string(10)
     assert mb.STATUS_NAMES[10] == "MUON_ERR_BOUNDS"
+
+
+def test_checkpoint_average_betas_match_the_oracle():
+    import oracle
+    w = [0.5, 1.0, 3.0, 2.0, 1.5, 4.0]
+    assert mb.checkpoint_average_betas(w) == pytest.approx(oracle.weighted_average_betas(w),
+                                                           rel=0, abs=1e-15)
+    assert mb.checkpoint_average_betas([2.0, 0.0, 1.0])[1] == 1.0  # zero weight: skip the call
+    with pytest.raises(ValueError):
+        mb.checkpoint_average_betas([0.0, 1.0])
+    with pytest.raises(ValueError):
+        mb.checkpoint_average_betas([1.0, -1.0])

@@ -33,3 +33,21 @@ def test_config_names_the_workload_and_its_cache_regime(wid):
     assert c["workload"] and c["banks"] and c["params"] == sum(b.count * b.rows * b.cols for b in w.banks)
     assert ("larger than L2" in c["l2"]) == (wid != 1)   # only the single 256x512 matrix fits in L2
     assert bench.launches_per_step(w) == 4
+
+
+def test_traffic_is_null_once_the_kernel_sources_change(monkeypatch):
+    sha = bench.kernel_source_sha16()
+    monkeypatch.setitem(bench.NS_CHAIN_TRAFFIC, 2, {"bytes": 1.0e9, "source_sha16": sha,
+                                                    "capture": "one chain launch"})
+    assert bench.chain_traffic(2) == (1.0e9, "one chain launch")
+    monkeypatch.setitem(bench.NS_CHAIN_TRAFFIC, 2, {"bytes": 1.0e9, "source_sha16": "0" * 16,
+                                                    "capture": "one chain launch"})
+    assert bench.chain_traffic(2)[0] is None
+    assert bench.chain_traffic(77)[0] is None
+
+
+def test_roofline_fraction_is_of_the_burst_peak():
+    peaks = dict(hbm=6500.0, burst=1600.0, sustained=1400.0, src="measured")
+    r = bench._roofline(800.0, peaks, 1.0e12, 1.25, None, "none")
+    assert r["peak"] == 1600.0 and r["frac"] == 0.5
+    assert r["frac_of_sustained"] == pytest.approx(800.0 / 1400.0)

@@ -5,9 +5,14 @@ pass would; each group's step starts on a side stream as soon as its
 gradients are final. The result must be exactly one plain call of the
 library on every bank with the same gradients, eagerly and replayed from a
 CUDA graph that holds the backward pass and the overlapped step together.
+The first (eager) overlapped step is also checked against the CPU oracle:
+every momentum element, the parameter step of sampled matrices and, with
+fp32 parameters, the orthogonalised update and its singular values.
 """
 import pytest
 import torch
+
+from _oracle_checks import check_anvil_step, check_muon_step, hp_dict
 
 pytestmark = pytest.mark.gpu
 
@@ -16,9 +21,9 @@ SHAPES = [(4, 768, 768), (2, 768, 3072), (2, 3072, 768), (3, 512, 1024)]
 GROUPS = [[3], [1, 2], [0]]          # the order the backward pass finishes them
 
 
-def _setup(seed):
+def _setup(seed, dtype):
     g = torch.Generator(device=DEV).manual_seed(seed)
-    params = [(torch.randn(c, r, k, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    params = [(torch.randn(c, r, k, generator=g, device=DEV) * 0.02).to(dtype)
               for c, r, k in SHAPES]
     # per bank: activations and output gradients whose product is the weight gradient
     acts = [(torch.randn(c, 64, r, generator=g, device=DEV), torch.randn(c, 64, k, generator=g, device=DEV))
@@ -31,8 +36,9 @@ def _grad(acts, b, out):
     torch.bmm(x.transpose(1, 2), dy, out=out)   # [c, r, k] = x^T dy
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("variant", ["muon", "anvil"])
-def test_overlapped_step_equals_one_call_eager_and_in_a_graph(variant):
+def test_overlapped_step_equals_one_call_eager_and_in_a_graph(variant, dtype):
     import muon_newton_schulz_05_b200 as mb
     from muon_newton_schulz_05_b200.overlap import OverlappedStep
     if variant == "anvil":
@@ -49,7 +55,9 @@ def test_overlapped_step_equals_one_call_eager_and_in_a_graph(variant):
             out.append(mb.Bank(p, gr, m, torch.zeros_like(m) if variant == "anvil" else None))
         return out
 
-    params, acts = _setup(5)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    params, acts = _setup(5, tdt)
+    params0 = [p.clone() for p in params]
     grads = [torch.empty(c, r, k, device=DEV) for c, r, k in SHAPES]
     banks = banks_for(params, grads)
     ov = OverlappedStep([[banks[b] for b in grp] for grp in GROUPS], hp, variant=variant)
@@ -79,6 +87,16 @@ def test_overlapped_step_equals_one_call_eager_and_in_a_graph(variant):
     for a, r in zip(banks, r_banks):
         assert torch.equal(a.param, r.param)
         assert torch.equal(a.momentum, r.momentum)
+    # the first step against the oracle (zero momenta before it)
+    ohp = hp_dict(hp)
+    for b, bk in enumerate(banks):
+        picks = [0, SHAPES[b][0] - 1]
+        zero = torch.zeros(bk.momentum.shape)
+        if variant == "anvil":
+            check_anvil_step(params0[b], bk.param, grads[b], zero, bk.momentum, zero,
+                             bk.momentum_slow, ohp, picks, dtype)
+        else:
+            check_muon_step(params0[b], bk.param, grads[b], zero, bk.momentum, ohp, picks, dtype)
 
     graph = torch.cuda.CUDAGraph()    # backward + overlapped step in one graph
     s = torch.cuda.Stream()

@@ -153,7 +153,7 @@ def test_gpt124m_bank_ten_steps():
 
 def test_square_1024_bank_with_decay():
     w = mi.workloads()[3]
-    _muon_run(w, 3, {0, 2}, lambda b, n: [0, 37])
+    _muon_run(w, w.steps, {0, 12, w.steps - 1}, lambda b, n: [0, 37, n - 1])
 
 
 def test_sgd_form_momentum_flag():
@@ -364,6 +364,74 @@ def test_bounded_wait_timeout_is_reported_and_recovers():
     assert rel_fro(f64(out[0]), ref) < TOL_UPDATE
 
 
+def test_timeout_in_a_step_leaves_params_and_ema_unchanged():
+    """A bounded wait that runs out inside a step (the test hook withholds one
+    operand stage) is reported, and the step writes no parameter and no EMA;
+    the momenta advanced once (their pass runs before the chain). While the
+    status word holds the error, further steps change nothing at all; once
+    it is cleared, steps run again and match the oracle."""
+    w, banks = _small_bank()
+    ws = mb.alloc_workspace([b.shape for b in banks])
+    H = mb.Hparams.from_dict(dict(w.hp, ema_beta=0.99))
+    grads = [mi.make_grads(w, b, 0) for b in range(2)]
+    for bk, g in zip(banks, grads):
+        bk.grad = g.to(DEV)
+    p0 = [b.param.clone() for b in banks]
+    e0 = [b.ema.clone() for b in banks]
+    try:
+        mb.set_debug(1, 0.25)
+        mb.muon_step(banks, H, ws)
+        assert mb.device_status(ws) == 8
+    finally:
+        mb.set_debug(0, 0.0)
+    for b, bk in enumerate(banks):
+        assert torch.equal(bk.param, p0[b]) and torch.equal(bk.ema, e0[b])
+        Mref = oracle.momentum_update(np.zeros(bk.momentum.shape), f64(grads[b]), w.hp["mu"])
+        assert buffer_ok(f64(bk.momentum), Mref)[0]
+    m1 = [b.momentum.clone() for b in banks]
+    mb.muon_step(banks, H, ws)             # the error is still recorded: a no-op
+    assert mb.device_status(ws, clear=True) == 8
+    for b, bk in enumerate(banks):
+        assert torch.equal(bk.param, p0[b]) and torch.equal(bk.ema, e0[b])
+        assert torch.equal(bk.momentum, m1[b])
+    mb.muon_step(banks, H, ws)             # cleared: a normal step
+    torch.cuda.synchronize()
+    assert mb.device_status(ws) == 0
+    for b, bk in enumerate(banks):
+        R, C = bk.shape[1:]
+        G = f64(grads[b][0])
+        Mref = oracle.momentum_update(f64(m1[b][0]), G, w.hp["mu"])
+        U = oracle.nesterov_lookahead(Mref, G, w.hp["mu"], True)
+        O = oracle.orthogonalize(U, w.hp["coeffs"], w.hp["eps"])
+        t0 = f64(p0[b][0])
+        dref = oracle.decoupled_update(t0, O, w.hp["lr"], w.hp["weight_decay"],
+                                       oracle.shape_scale(R, C)) - t0
+        ok, r = delta_ok(t0, f64(bk.param[0]), dref, "bf16")
+        assert ok, r
+
+
+def test_weighted_checkpoint_average_through_ema_update():
+    """Weighted checkpoint average ("qlabs-eng/slowrun", leaderboard: weighted
+    checkpoint averaging) as ema_update with the running beta of each
+    checkpoint, against the oracle's sum w_i theta_i / sum w_i."""
+    n, shape = 7, (3, 129, 200)
+    weights = [0.5, 1.0, 3.0, 0.0, 2.0, 1.5, 4.0]
+    thetas = [mi.gaussian(shape[0] * shape[1], shape[2], 500 + i, 0.02).reshape(shape)
+              .to(torch.bfloat16) for i in range(n)]
+    th = thetas[0].to(DEV)
+    avg = torch.zeros(shape, device=DEV)
+    bank = mb.Bank(th, th, torch.zeros(shape, device=DEV), None, avg)
+    for wt, w_i, beta in zip(thetas, weights, mb.checkpoint_average_betas(weights)):
+        if w_i == 0.0:
+            continue  # no weight: the checkpoint does not enter the average
+        th.copy_(wt.to(DEV))
+        mb.ema_update([bank], beta)
+    torch.cuda.synchronize()
+    ref = oracle.weighted_average([f64(t) for t in thetas], weights)
+    ok, r = buffer_ok(f64(avg), ref)
+    assert ok, r
+
+
 def test_invalid_arguments_launch_nothing():
     x = torch.zeros(1, 64, 64, dtype=torch.bfloat16, device=DEV)
     ws = torch.zeros(16, dtype=torch.uint8, device=DEV)
@@ -405,3 +473,9 @@ def test_transformer_2p5b_bank_sampled():
                                            oracle.shape_scale(R, C)) - t0
             ok, r = delta_ok(t0, f64(bk.param[i]), dref, "bf16")
             assert ok, ("delta", b, i, r)
+            # the Newton-Schulz chain at this size on the same U (one matrix,
+            # the benchmark's kernel): relative Frobenius and singular values
+            Ug = torch.from_numpy(U.astype(np.float32))[None].to(DEV)
+            Og = f64(orth_gpu(Ug, hp["coeffs"])[0])
+            assert rel_fro(Og, O) <= TOL_UPDATE, ("O", b, i, rel_fro(Og, O))
+            assert sv_maxdiff(Og, O) <= TOL_SV, ("singular values", b, i)
