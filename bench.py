@@ -13,6 +13,14 @@ step, phase and matrix) -> scaled parameter write.
 The same run also times the 64 x 1024^2 bank (20 steps after 3 warm-up
 steps) for its Newton-Schulz roofline line.
 `--impl reference` times the CPU oracle (host cores) on the whole bank.
+
+N > 1 (under torchrun, one process per GPU) is data-parallel training's
+optimizer step: every rank holds the same bank and its own gradient; the
+ranks average the gradients with a reduce-scatter, each steps the matrices
+it owns, and an all-gather brings every rank the updated bank (the bank
+storage is laid out in owner order, so nothing is packed or unpacked). The
+total work is one bank step however many GPUs share it (strong scaling);
+`--mode replica` instead gives every rank its own bank (weak scaling).
 """
 from __future__ import annotations
 
@@ -57,6 +65,8 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-square", action="store_true",
                     help="skip the 64 x 1024^2 roofline line")
+    ap.add_argument("--mode", default="sharded", choices=["sharded", "replica"],
+                    help="N > 1: data-parallel owner-sharded step (default) or one bank per rank")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
                     help="1..5 (default 2, the GPT-124M bank the metric names); the others "
                          "are measured for documentation only")
@@ -110,7 +120,7 @@ def _ns_flops(w) -> float:
     return tot
 
 
-def _config(w, extra=None):
+def _config(w, extra=None, parallelism="replica per GPU (independent banks)"):
     names = {1: "single_256x512_fp32", 2: "gpt124m_matrix_bank", 3: "square_1024x1024x64_bank",
              4: "transformer_2p5b_matrix_bank", 5: "anvil_gpt124m_bank_plus_readout"}
     if w.variant == "anvil":
@@ -127,7 +137,7 @@ def _config(w, extra=None):
          "grads": f"N(0,{w.grad_sigma:g}^2)" + (f" + rank-{w.spike_rank} spike at 10x RMS" if w.spike_rank else ""),
          "l2": (f"inputs larger than L2: ~{touched:.2f} GB touched per step (126 MB L2), no flush"
                 if touched > 0.126 else f"~{touched*1e3:.0f} MB touched per step: fits in L2, no flush"),
-         "parallelism": "replica per GPU (independent banks)"}
+         "parallelism": parallelism}
     if extra:
         c.update(extra)
     return c
@@ -521,10 +531,143 @@ def _square_roofline(args, dev, peaks, steps=20, warmup=3):
     return r
 
 
+def run_sharded(args):
+    """N ranks share one data-parallel optimizer step of the bank."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import muon_inputs as mi
+    import muon_newton_schulz_05_b200 as mb
+    from muon_newton_schulz_05_b200.sharded import ShardedBankMuon
+
+    world = int(os.environ["WORLD_SIZE"])
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = _workload(args.workload)
+    peaks = _peaks()
+    anvil = w.variant == "anvil"
+    shapes = [(b.count, b.rows, b.cols) for b in w.banks]
+    opt = ShardedBankMuon(shapes, mi.torch_dtype(w.param_dtype), mi.torch_dtype(w.grad_dtype),
+                          variant=w.variant, device=dev, ema=anvil)
+    host_grads = []
+    for b in range(len(w.banks)):
+        opt.params[b].copy_(mi.make_params(w, b).to(dev))   # the same bank on every rank
+        g = mi.make_grads(w, b, rank)                         # this rank's own gradient
+        host_grads.append(g.pin_memory())
+        opt.grads[b].copy_(g.to(dev))
+    H = mb.Hparams.from_dict(w.hp)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        opt.step(H)
+    torch.cuda.synchronize()
+    assert opt.workspace is None or mb.device_status(opt.workspace) == 0
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize()
+    t_begin.record(stream)
+    for s_ in range(K):
+        mb.set_ns_events(ev[2 * s_], ev[2 * s_ + 1])
+        opt.step(H)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    mb.set_ns_events(None, None)
+    step_ms = t_begin.elapsed_time(t_end)
+    total_ms = max_over_ranks(step_ms, dist, dev)
+    owned = opt.owned_shapes()
+    ns_ms = statistics.mean(ev[2 * s_].elapsed_time(ev[2 * s_ + 1]) for s_ in range(K)) if owned else 0.0
+
+    # the same owner step without the exchange (this rank's matrices only)
+    local_ms = 0.0
+    if owned:
+        banks = [mb.Bank(opt.params[b][lo:hi], opt.grads[b][lo:hi], opt.momentum[b],
+                         opt.momentum_slow[b], opt.ema[b])
+                 for b, (lo, hi) in enumerate(opt.owned) if hi > lo]
+        fn = mb.anvil_step if anvil else mb.muon_step
+        l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        l0.record(stream)
+        for _ in range(K):
+            fn(banks, H, opt.workspace)
+        l1.record(stream)
+        torch.cuda.synchronize()
+        local_ms = l0.elapsed_time(l1) / K
+    local_max = max_over_ranks(local_ms, dist, dev)
+
+    # end to end: this rank's gradients in from pinned host memory and the
+    # updated bank out, every step, on the step's stream
+    host_params = [torch.empty(p.shape, dtype=p.dtype).pin_memory() for p in opt.params]
+    E = args.e2e_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(E):
+        for g, hg in zip(opt.grads, host_grads):
+            g.copy_(hg, non_blocking=True)
+        opt.step(H)
+        for hp_, p in zip(host_params, opt.params):
+            hp_.copy_(p, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    h2d = sum(g.numel() * g.element_size() for g in host_grads)
+    d2h = sum(p.numel() * p.element_size() for p in host_params)
+    assert opt.workspace is None or mb.device_status(opt.workspace) == 0
+
+    my_flops = 0.0
+    k = len(w.hp["coeffs"])
+    for c, r_, c_ in owned:
+        rr, cc = min(r_, c_), max(r_, c_)
+        my_flops += c * k * (rr * (rr + 1) * cc + rr * rr * (rr + 1) + 2.0 * rr * rr * cc)
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    achieved = my_flops / (ns_ms * 1e-3) / 1e12 if ns_ms > 0 else 0.0
+    roof = _roofline(achieved, peaks, my_flops, ns_ms, None,
+                     "no ncu capture of a multi-rank run (ncu runs on one GPU only)")
+    roof["kernel"] = "ns_gemm_kernel on rank 0's owned matrices"
+    line = {
+        "metric": METRIC, "value": K / (total_ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(w, parallelism=f"dp{world}: owner-sharded data-parallel step "
+                                         "(reduce-scatter, owner step, all-gather; NCCL)"),
+        "roofline": roof,
+        "sharded": {"owned_shapes_rank0": owned, "load_max_over_mean":
+                    max(opt.layout.load) / (sum(opt.layout.load) / world),
+                    "local_step_ms_max": local_max, "exchange_ms": total_ms / K - local_max},
+        "cpu_baseline": None,
+        "e2e": {"value": E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "what": "per step and rank: pinned host->device copy of the rank's gradients, "
+                        "the sharded step, device->host copy of the updated bank"},
+        "gpu_launches": launches_per_step(w) * K,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = _args()
     if args.impl == "reference":
         return run_reference(args)
+    # under torchrun (any N, one included) the data-parallel sharded step;
+    # a plain `python bench.py` is the single-GPU bank step
+    if "WORLD_SIZE" in os.environ and args.mode == "sharded":
+        return run_sharded(args)
     return run_native(args)
 
 

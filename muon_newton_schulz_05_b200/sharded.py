@@ -310,3 +310,235 @@ class ShardedMuon:
             else:
                 self.dist.all_gather_into_tensor(flat, seg, group=self.group)
             self.plan.unpack(k, flat, out)
+
+
+# ---------------------------------------------------------------------------
+# Owner-ordered bank storage: the same step without any packing copies
+# ---------------------------------------------------------------------------
+@dataclass
+class BankSlots:
+    """Where one bank lives in its owner-ordered buffer. The buffer holds
+    world * seg matrix slots; rank r owns slots [r seg, (r + 1) seg); the
+    bank's count matrices fill slots [offset, offset + count) in order, the
+    rest is padding."""
+    count: int
+    seg: int
+    offset: int
+
+    def owned(self, rank: int) -> Tuple[int, int]:
+        """Matrices [lo, hi) of the bank that rank owns (lo == hi: none)."""
+        lo = max(rank * self.seg, self.offset) - self.offset
+        hi = min((rank + 1) * self.seg, self.offset + self.count) - self.offset
+        return lo, max(lo, hi)
+
+
+@dataclass
+class OwnerLayout:
+    world: int
+    shapes: List[Tuple[int, int, int]]
+    banks: List[BankSlots]
+    load: List[float]                # per-rank Newton-Schulz work
+
+    @classmethod
+    def build(cls, shapes: Sequence[Tuple[int, int, int]], world: int) -> "OwnerLayout":
+        """Each bank gets ceil(count / world) slots per rank, so every rank owns
+        a contiguous run of its matrices; the bank's offset in the buffer (how
+        many padding slots come first) is chosen, heaviest banks first, to
+        keep the ranks' Newton-Schulz work (3 r^2 c + r^3 per matrix) as even
+        as the contiguous runs allow."""
+        shapes = [tuple(int(v) for v in s) for s in shapes]
+        if world < 1:
+            raise ValueError("world size must be >= 1")
+        load = [0.0] * world
+        slots: List[Optional[BankSlots]] = [None] * len(shapes)
+        order = sorted(range(len(shapes)), key=lambda b: (-ns_work(shapes[b][1], shapes[b][2]), b))
+        for b in order:
+            count, rows, cols = shapes[b]
+            seg = -(-count // world)
+            w = ns_work(rows, cols)
+            best = None
+            for off in range(world * seg - count + 1):
+                cand = BankSlots(count, seg, off)
+                new = [load[r] + w * (lambda lh: lh[1] - lh[0])(cand.owned(r)) for r in range(world)]
+                key = (max(new), sum(x * x for x in new), off)
+                if best is None or key < best[0]:
+                    best = (key, cand, new)
+            slots[b] = best[1]
+            load = best[2]
+        return cls(world, shapes, slots, load)
+
+    def signature(self) -> Tuple:
+        return (self.world, tuple(self.shapes),
+                tuple((s.count, s.seg, s.offset) for s in self.banks))
+
+
+class ShardedBankMuon:
+    """Owner-sharded data-parallel Muon (or ANVIL) step on bank storage that the
+    optimizer owns, laid out in owner order (see OwnerLayout): no gradient is
+    packed and no parameter is unpacked.
+
+    `params[b]` and `grads[b]` are this rank's [count, R, C] bank tensors,
+    views into one flat buffer per bank: load the model's weights into
+    `params` (identical on every rank) and let the backward pass write this
+    rank's gradients into `grads`. One step: an averaging reduce-scatter of
+    every bank's gradient buffer in place (each rank receives its own slots);
+    the optimizer step (the CUDA library, one call over all banks) on the
+    matrices this rank owns, in place; an all-gather of every parameter
+    buffer in place. Momenta (and the EMA) exist only for the owned matrices.
+    A training loop may call `grad_ready(b)` as soon as bank b's gradients
+    are final, then `finish(hp)`; `step(hp)` does both.
+    Requires rows * cols to be a multiple of 8, so that every matrix slot
+    starts on a 16-byte boundary.
+    """
+
+    def __init__(self, shapes, param_dtype, grad_dtype, group=None, variant: str = "muon",
+                 device=None, ema: bool = False, step_fn: Optional[Callable] = None,
+                 workspace_fn: Optional[Callable] = None):
+        import torch
+        import torch.distributed as dist
+        if variant not in ("muon", "anvil"):
+            raise ValueError("variant must be 'muon' or 'anvil'")
+        shapes = [tuple(int(v) for v in s) for s in shapes]
+        for c, r, k in shapes:
+            if (r * k) % 8:
+                raise ValueError(f"rows * cols of a {r} x {k} matrix is not a multiple of 8")
+        self.dist, self.group = dist, group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.gloo = dist.get_backend(group) == "gloo"
+        self.layout = OwnerLayout.build(shapes, self.world)
+        self.variant = variant
+        self.device = device if device is not None else torch.device("cpu")
+        if step_fn is None or workspace_fn is None:
+            from . import alloc_workspace, anvil_step, muon_step
+            step_fn = step_fn or (anvil_step if variant == "anvil" else muon_step)
+            workspace_fn = workspace_fn or (lambda shapes: alloc_workspace(shapes, self.device))
+        self.step_fn, self.workspace_fn = step_fn, workspace_fn
+        self._pflat, self._gflat = [], []
+        self.params, self.grads = [], []
+        self.momentum, self.momentum_slow, self.ema = [], [], []
+        self.owned = []
+        for (count, rows, cols), sl in zip(shapes, self.layout.banks):
+            rc = rows * cols
+            n = self.world * sl.seg * rc
+            pf = torch.zeros(n, dtype=param_dtype, device=self.device)
+            gf = torch.zeros(n, dtype=grad_dtype, device=self.device)
+            self._pflat.append(pf)
+            self._gflat.append(gf)
+            self.params.append(pf[sl.offset * rc:(sl.offset + count) * rc].view(count, rows, cols))
+            self.grads.append(gf[sl.offset * rc:(sl.offset + count) * rc].view(count, rows, cols))
+            lo, hi = sl.owned(self.rank)
+            self.owned.append((lo, hi))
+
+            def state(on):
+                if not on or hi == lo:
+                    return None
+                return torch.zeros(hi - lo, rows, cols, dtype=torch.float32, device=self.device)
+            self.momentum.append(state(True))
+            self.momentum_slow.append(state(variant == "anvil"))
+            self.ema.append(state(ema))
+        self.workspace = None
+        self._ema_ready = False
+        self._pending: List = [None] * len(shapes)
+
+    def _segment(self, flat, b):
+        sl = self.layout.banks[b]
+        rc = self.layout.shapes[b][1] * self.layout.shapes[b][2]
+        return flat[self.rank * sl.seg * rc:(self.rank + 1) * sl.seg * rc]
+
+    def owned_shapes(self) -> List[Tuple[int, int, int]]:
+        return [(hi - lo, s[1], s[2]) for (lo, hi), s in zip(self.owned, self.layout.shapes)
+                if hi > lo]
+
+    def grad_ready(self, b: int) -> None:
+        """Bank b's gradients in `grads[b]` are final: start their averaging
+        reduce-scatter (in place: this rank's slots receive the mean)."""
+        if self._pending[b] is not None:
+            raise RuntimeError(f"bank {b} is already in flight in this step")
+        flat, seg = self._gflat[b], self._segment(self._gflat[b], b)
+        if self.gloo:
+            # gloo has no reduce-scatter: sum everywhere, scale this rank's slots
+            self.dist.all_reduce(flat, op=self.dist.ReduceOp.SUM, group=self.group)
+            seg.div_(self.world)
+            self._pending[b] = True
+        else:
+            self._pending[b] = self.dist.reduce_scatter_tensor(
+                seg, flat, op=self.dist.ReduceOp.AVG, group=self.group, async_op=True)
+
+    def finish(self, hp) -> None:
+        """Step the owned matrices of every bank (all must be grad_ready) with
+        one library call, then all-gather every parameter buffer in place."""
+        from . import Bank
+        if any(w is None for w in self._pending):
+            raise RuntimeError("every bank needs grad_ready before finish")
+        for w in self._pending:
+            if w is not True:
+                w.wait()
+        banks = []
+        for b, (lo, hi) in enumerate(self.owned):
+            if hi == lo:
+                continue
+            p, g = self.params[b][lo:hi], self.grads[b][lo:hi]
+            if self.ema[b] is not None and not self._ema_ready:
+                self.ema[b].copy_(p)  # the average starts at the parameters it averages
+            banks.append(Bank(p, g, self.momentum[b], self.momentum_slow[b], self.ema[b]))
+        if banks:
+            if self.workspace is None:
+                self.workspace = self.workspace_fn([bk.shape for bk in banks])
+            self.step_fn(banks, hp, self.workspace)
+        works = []
+        for b in range(len(self.layout.banks)):
+            flat, seg = self._pflat[b], self._segment(self._pflat[b], b)
+            if self.gloo:
+                self.dist.all_gather(list(flat.chunk(self.world)), seg.clone(), group=self.group)
+            else:
+                works.append(self.dist.all_gather_into_tensor(flat, seg, group=self.group,
+                                                              async_op=True))
+        for w in works:
+            w.wait()
+        self._pending = [None] * len(self.layout.banks)
+        self._ema_ready = True
+
+    def step(self, hp) -> None:
+        for b in range(len(self.layout.banks)):
+            self.grad_ready(b)
+        self.finish(hp)
+
+    def state_dict(self) -> dict:
+        def cpu(ts):
+            return [t.detach().cpu().clone() if t is not None else None for t in ts]
+        return {"layout": self.layout.signature(), "rank": self.rank, "variant": self.variant,
+                "momentum": cpu(self.momentum), "momentum_slow": cpu(self.momentum_slow),
+                "ema": cpu(self.ema), "ema_ready": self._ema_ready}
+
+    def load_state_dict(self, state: dict) -> None:
+        if state["layout"] != self.layout.signature() or state["rank"] != self.rank:
+            raise ValueError("the state was saved under another layout or rank")
+        if state["variant"] != self.variant:
+            raise ValueError("the state was saved by the other variant")
+        for name in ("momentum", "momentum_slow", "ema"):
+            for t, v in zip(getattr(self, name), state[name]):
+                if (t is None) != (v is None):
+                    raise ValueError(f"{name}: the saved state has a different layout")
+                if t is not None:
+                    t.copy_(v)
+        self._ema_ready = bool(state["ema_ready"])
+
+    def gather_ema(self, out: Sequence) -> None:
+        """Collect the owners' EMA of every matrix into out (fp32 bank tensors)."""
+        import torch
+        for b, ((count, rows, cols), sl) in enumerate(zip(self.layout.shapes, self.layout.banks)):
+            rc = rows * cols
+            flat = torch.zeros(self.world * sl.seg * rc, dtype=torch.float32, device=self.device)
+            seg = self._segment(flat, b)
+            lo, hi = self.owned[b]
+            if hi > lo:
+                if self.ema[b] is None:
+                    raise RuntimeError("ShardedBankMuon was built without ema=True")
+                start = (max(self.rank * sl.seg, sl.offset) - self.rank * sl.seg) * rc
+                seg[start:start + (hi - lo) * rc].copy_(self.ema[b].reshape(-1))
+            if self.gloo:
+                self.dist.all_gather(list(flat.chunk(self.world)), seg.clone(), group=self.group)
+            else:
+                self.dist.all_gather_into_tensor(flat, seg, group=self.group)
+            out[b].copy_(flat[sl.offset * rc:(sl.offset + count) * rc].view(count, rows, cols))

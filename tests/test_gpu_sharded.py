@@ -102,3 +102,54 @@ def test_sharded_single_rank_equals_direct_step_and_oracle(nccl_group, variant, 
         opt.gather_ema(out)
         for b in range(3):
             assert torch.equal(out[b], ema[b])
+
+
+@pytest.mark.parametrize("variant", ["muon", "anvil"])
+def test_bank_storage_single_rank_equals_direct_step_and_oracle(nccl_group, variant):
+    """ShardedBankMuon (owner-ordered bank storage, in-place reduce-scatter and
+    all-gather) on one rank: bitwise a direct call of the library, and the
+    oracle on the second step (fp32 parameters: O recovered from the step)."""
+    import muon_newton_schulz_05_b200 as mb
+    from muon_newton_schulz_05_b200.sharded import ShardedBankMuon
+    hp = _hparams(variant)
+    ohp = hp_dict(hp)
+    opt = ShardedBankMuon(SHAPES, torch.float32, torch.bfloat16, variant=variant, device=DEV,
+                          ema=(variant == "anvil"))
+    init = _bank(2, 0.02)
+    for p, p0 in zip(opt.params, init):
+        p.copy_(p0)
+    ref = [p.clone() for p in init]
+    mom = [torch.zeros(c, r, k, device=DEV) for c, r, k in SHAPES]
+    slow = [torch.zeros_like(m) for m in mom] if variant == "anvil" else [None] * 3
+    ema = [p.clone() for p in ref] if variant == "anvil" else [None] * 3
+    banks = [mb.Bank(ref[b], None, mom[b], slow[b], ema[b]) for b in range(3)]
+    ws = mb.alloc_workspace([bk.shape for bk in banks])
+    for s in range(3):
+        grads = [g.to(torch.bfloat16) for g in _bank(200 + s)]
+        for g, g0 in zip(opt.grads, grads):
+            g.copy_(g0)
+        before = [(p.clone(), m.clone(), None if sl is None else sl.clone())
+                  for p, m, sl in zip(opt.params, mom, slow)]
+        opt.step(hp)
+        for b in range(3):
+            banks[b].grad = grads[b]
+        (mb.anvil_step if variant == "anvil" else mb.muon_step)(banks, hp, ws)
+        torch.cuda.synchronize()
+        for b in range(3):
+            assert torch.equal(opt.params[b], ref[b]), (s, b)
+            assert torch.equal(opt.momentum[b], mom[b])
+        if s == 1:
+            for b in range(3):
+                picks = [0, SHAPES[b][0] - 1]
+                th0, m0, sl0 = before[b]
+                if variant == "anvil":
+                    check_anvil_step(th0, opt.params[b], grads[b], m0, mom[b], sl0, slow[b], ohp,
+                                     picks, "f32")
+                else:
+                    check_muon_step(th0, opt.params[b], grads[b], m0, mom[b], ohp, picks, "f32")
+    assert mb.device_status(ws) == 0 and mb.device_status(opt.workspace) == 0
+    if variant == "anvil":
+        out = [torch.zeros(c, r, k, device=DEV) for c, r, k in SHAPES]
+        opt.gather_ema(out)
+        for b in range(3):
+            assert torch.equal(out[b], ema[b])

@@ -334,3 +334,150 @@ def test_plan_rejects_bad_buckets():
         ShardPlan.build(SHAPES, 2, [[0, 1], [1, 2]])
     with pytest.raises(ValueError):
         ShardPlan.build(SHAPES, 0)
+
+
+# ---------------------------------------------------------------------------
+# Owner-ordered bank storage (ShardedBankMuon): no packing copies
+# ---------------------------------------------------------------------------
+from muon_newton_schulz_05_b200.sharded import OwnerLayout  # noqa: E402
+
+
+def _bank_rank_main(rank, world, port, variant, steps, order, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from muon_newton_schulz_05_b200.sharded import ShardedBankMuon
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        opt = ShardedBankMuon(SHAPES, torch.bfloat16, torch.float32, variant=variant,
+                              ema=(variant == "anvil"), step_fn=_oracle_step_fn(variant),
+                              workspace_fn=lambda shapes: None)
+        for p, p0 in zip(opt.params, _params(SHAPES)):
+            p.copy_(p0)
+        hp = _hparams(variant)
+        for s in range(steps):
+            for g, g0 in zip(opt.grads, _grads(SHAPES, rank, s)):
+                g.copy_(g0)
+            for b in order:            # the order the backward pass finishes the banks
+                opt.grad_ready(b)
+            opt.finish(hp)
+        res = {"params": [p.float().numpy().copy() for p in opt.params],
+               "owned": list(opt.owned)}
+        if variant == "anvil":
+            ema = [torch.zeros(c, r, k) for c, r, k in SHAPES]
+            opt.gather_ema(ema)
+            res["ema"] = [e.numpy() for e in ema]
+        out[rank] = res
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("variant,world,order", [("muon", 2, [0, 1, 2]), ("anvil", 2, [2, 1, 0]),
+                                                 ("muon", 3, [1, 0, 2])])
+def test_bank_storage_step_equals_single_process_step(variant, world, order):
+    """Every rank ends with the bank one process gets by stepping every matrix
+    on the mean of the ranks' gradients (gradients summed in the same order on
+    both sides for two ranks; three ranks use integer-exact sums below)."""
+    port = _free_port()
+    steps = 2
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_bank_rank_main, args=(world, port, variant, steps, order, out), nprocs=world,
+                 join=True)
+        res = dict(out)
+    # every matrix owned by exactly one rank
+    for b, (count, _, _) in enumerate(SHAPES):
+        got = sorted(i for r in range(world) for i in range(*res[r]["owned"][b]))
+        assert got == list(range(count))
+    if world == 2:
+        ref_params, ref_ema = _single_process(variant, steps, world)
+        for b in range(len(SHAPES)):
+            for r in range(world):
+                np.testing.assert_array_equal(res[r]["params"][b], ref_params[b].float().numpy())
+                if variant == "anvil":
+                    np.testing.assert_array_equal(res[r]["ema"][b], ref_ema[b].numpy())
+    else:
+        # float sums over three ranks may round differently: every rank agrees,
+        # and each matches the single-process step closely
+        from muon_newton_schulz_05_b200 import Bank
+        params = _params(SHAPES)
+        mom = [torch.zeros(c, r, k) for c, r, k in SHAPES]
+        step = _oracle_step_fn("muon")
+        for s in range(steps):
+            gs = [_grads(SHAPES, r, s) for r in range(world)]
+            mean = [sum(g[b] for g in gs) / world for b in range(len(SHAPES))]
+            step([Bank(params[b], mean[b], mom[b]) for b in range(len(SHAPES))], _hparams("muon"), None)
+        for b in range(len(SHAPES)):
+            for r in range(1, world):
+                np.testing.assert_array_equal(res[r]["params"][b], res[0]["params"][b])
+            np.testing.assert_allclose(res[0]["params"][b], params[b].float().numpy(),
+                                       rtol=0, atol=2e-2 * np.abs(params[b].float().numpy()).max())
+
+
+def test_owner_layout_covers_every_matrix_and_balances():
+    for world in (1, 2, 3, 4, 8):
+        lay = OwnerLayout.build(GPT_SHAPES, world)
+        total = sum(c * ns_work(r, k) for c, r, k in GPT_SHAPES)
+        assert abs(sum(lay.load) - total) < 1e-6 * total
+        for (count, _, _), sl in zip(GPT_SHAPES, lay.banks):
+            runs = [sl.owned(r) for r in range(world)]
+            assert [i for lo, hi in runs for i in range(lo, hi)] == list(range(count))
+            assert sl.offset + count <= world * sl.seg and sl.seg == -(-count // world)
+        # divisible counts split evenly; 12 large matrices over 8 ranks cannot
+        if world in (1, 2, 3, 4):
+            assert max(lay.load) == pytest.approx(total / world, rel=1e-12)
+        else:
+            assert max(lay.load) <= 1.25 * total / world
+    with pytest.raises(ValueError):
+        OwnerLayout.build(GPT_SHAPES, 0)
+
+
+def _bank_resume_rank(rank, world, port, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from muon_newton_schulz_05_b200.sharded import ShardedBankMuon
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        def make():
+            o = ShardedBankMuon(SHAPES, torch.bfloat16, torch.float32, variant="anvil", ema=True,
+                                step_fn=_oracle_step_fn("anvil"), workspace_fn=lambda shapes: None)
+            for p, p0 in zip(o.params, _params(SHAPES)):
+                p.copy_(p0)
+            return o
+        hp = _hparams("anvil")
+
+        def run(o, steps):
+            for s in steps:
+                for g, g0 in zip(o.grads, _grads(SHAPES, rank, s)):
+                    g.copy_(g0)
+                o.step(hp)
+        a = make()
+        run(a, range(4))
+        b = make()
+        run(b, range(2))
+        saved = b.state_dict()
+        c = make()
+        for p, q in zip(c.params, b.params):   # the weights come from the model checkpoint
+            p.copy_(q)
+        c.load_state_dict(saved)
+        run(c, range(2, 4))
+        same = all(torch.equal(x, y) for x, y in zip(a.params, c.params))
+        ea = [torch.zeros(cc, r, k) for cc, r, k in SHAPES]
+        ec = [torch.zeros(cc, r, k) for cc, r, k in SHAPES]
+        a.gather_ema(ea)
+        c.gather_ema(ec)
+        out[rank] = (same, all(torch.equal(x, y) for x, y in zip(ea, ec)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bank_storage_state_resumes_bitwise():
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_bank_resume_rank, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[0] == (True, True) and res[1] == (True, True), res
