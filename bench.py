@@ -514,6 +514,8 @@ def _square_roofline(args, dev, peaks, steps=20, warmup=3):
     for _ in range(warmup):
         mb.muon_step(banks, H, ws)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+    for e in ev:  # torch creates the event handles lazily: make them exist
+        e.record(stream)
     torch.cuda.synchronize()
     for s_ in range(steps):
         mb.set_ns_events(ev[2 * s_], ev[2 * s_ + 1])
@@ -567,6 +569,8 @@ def run_sharded(args):
 
     K = args.steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K)]
+    for e in ev:  # torch creates the event handles lazily: make them exist
+        e.record(stream)
     t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = Clocks(local)
     clocks.start()

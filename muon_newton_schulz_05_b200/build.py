@@ -41,8 +41,11 @@ def needs_build(lib: str = LIB) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, check: bool = False) -> str:
-    lib = LIB_CHECK if check else LIB
+def build(force: bool = False, ptxas_verbose: bool = False, check: bool = False,
+          out: str = None, defines=()) -> str:
+    """Compile the library. out/defines build a variant elsewhere (tuning
+    constants such as MUON_STAGES=5) without touching the in-tree library."""
+    lib = out or (LIB_CHECK if check else LIB)
     if not force and not needs_build(lib):
         return lib
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
@@ -50,6 +53,7 @@ def build(force: bool = False, ptxas_verbose: bool = False, check: bool = False)
            "-I", INCLUDE, "-I", CSRC, "-o", lib + ".tmp"]
     if check:
         cmd += ["-DMUON_CHECK"]
+    cmd += [f"-D{d}" for d in defines]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
@@ -64,4 +68,8 @@ def build(force: bool = False, ptxas_verbose: bool = False, check: bool = False)
 
 
 if __name__ == "__main__":
-    print(build(force=True, ptxas_verbose="--verbose-ptxas" in sys.argv, check="--check" in sys.argv))
+    args = sys.argv[1:]
+    out = args[args.index("--out") + 1] if "--out" in args else None
+    defines = [a[2:] for a in args if a.startswith("-D")]
+    print(build(force=True, ptxas_verbose="--verbose-ptxas" in args, check="--check" in args,
+                out=out, defines=defines))

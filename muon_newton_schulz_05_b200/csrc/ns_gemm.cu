@@ -255,33 +255,51 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_majo
 // ---------------------------------------------------------------- epilogues
 // Each epilogue warp owns 32 accumulator rows and 128 of the 256 columns and
 // works through them in 32 x 32 chunks. Global traffic goes through TMA only,
-// through kEpiBufs chunk buffers per warp: the bulk loads of a tile's first
-// chunks (Apply: hi and lo of the iterate; Poly: A) are issued when the tile
-// starts, and the stores of earlier chunks drain while later ones are
-// computed. Halves use the 64-byte swizzle of the TMA box (16-byte group g of
+// through kEpiBufs chunk buffers per warp: the bulk loads of the chunks' inputs
+// (Apply: hi and lo of the iterate; Poly: A) run kEpiBufs chunks ahead, across
+// tile boundaries, and the stores of earlier chunks drain while later ones
+// are computed. Halves use the 64-byte swizzle of the TMA box (16-byte group g of
 // row r at r*64 + ((g ^ ((r >> 1) & 3)) * 16)), so a lane reading or writing
 // its own row touches 8 distinct bank groups per quarter warp.
 __device__ __forceinline__ uint32_t swz64_off(int r, int g) {
   return static_cast<uint32_t>(r * 64 + ((g ^ ((r >> 1) & 3)) << 4));
 }
 
+// Ring positions: every chunk this warp handles takes the next position k;
+// position k uses buffer k % kEpiBufs and load barrier k % kEpiBufs. A load
+// for position k is issued once position k - kEpiBufs has had its store read
+// out of the buffer, so it may be issued up to kEpiBufs positions early, also
+// for the first chunks of the warp's next tile (loads run across tiles).
 struct EpiRing {
   uint8_t* base;     // kEpiBufs buffers of kEpiChunkBytes (two halves each)
   uint64_t* bar;     // kEpiBufs load barriers
   uint32_t parity;   // bit i: parity of the next completion of bar[i]
   uint32_t chunk;    // chunks handled so far by this warp (ring position)
+  uint32_t inflight; // lane 0: bit i set while a load into buffer i is outstanding
 };
 
 __device__ __forceinline__ uint8_t* ring_buf(const EpiRing& e, uint32_t k) {
   return e.base + (k % kEpiBufs) * kEpiChunkBytes;
 }
 
+// The epilogue of Apply (hi and lo of the iterate) and Poly (A) tiles reads
+// inputs; Gram tiles only store.
+__device__ __forceinline__ bool epi_has_loads(const Tile& T) {
+  return T.phase == kApply || T.phase == kPoly;
+}
+
+// Non-blocking: has the phase this tile reads finished (acquire, GPU scope)?
+__device__ __forceinline__ bool dependency_met(const Tile& T) {
+  return T.dep_target <= 0 || ld_acquire_gpu(T.dep_cnt) >= T.dep_target;
+}
+
 // Lane 0 issues the bulk loads of ring chunk k (column c0 of this warp's rows).
-__device__ __forceinline__ void epi_issue_load(const NsGemmParams& p, const EpiRing& e,
+__device__ __forceinline__ void epi_issue_load(const NsGemmParams& p, EpiRing& e,
                                                const Tile& T, const BankPlan& bp, int r0, int c0,
                                                uint32_t k) {
   uint8_t* b = ring_buf(e, k);
   uint64_t* bar = &e.bar[k % kEpiBufs];
+  e.inflight |= 1u << (k % kEpiBufs);
   if (T.phase == kApply) {
     const int y = T.mat * bp.Rp + r0;
     if (!in_bounds(T.mat < bp.count && r0 + kEpiRows <= bp.Rp && c0 + kEpiCols <= bp.Cp, p.status)) {
@@ -301,13 +319,39 @@ __device__ __forceinline__ void epi_issue_load(const NsGemmParams& p, const EpiR
   }
 }
 
-// Every lane waits for ring chunk k's loads. False if the wait gave up.
+// Chunk j (of kChunks) of tile X for this warp: lane 0 issues its loads into
+// ring position k.
+__device__ __forceinline__ void epi_issue_chunk(const NsGemmParams& p, EpiRing& e, const Tile& X,
+                                                int rank, int q, int half, int j, uint32_t k) {
+  const BankPlan& bp = p.bank[X.bank];
+  epi_issue_load(p, e, X, bp, X.m0 + kBM * rank + 32 * q, X.n0 + half * 128 + j * kEpiCols, k);
+}
+
+// Every lane waits for ring chunk k's loads. False if the wait gave up (the
+// load then still counts as outstanding, so that it can be drained).
 __device__ __forceinline__ bool epi_wait_load(const NsGemmParams& p, EpiRing& e, uint32_t k,
                                               volatile int* abort_flag) {
   const uint32_t i = k % kEpiBufs;
-  const bool ok = mbar_wait(&e.bar[i], (e.parity >> i) & 1u, abort_flag, p.status, p.wait_limit_ns);
-  e.parity ^= 1u << i;
-  return __all_sync(0xffffffffu, ok);
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&e.bar[i], (e.parity >> i) & 1u, abort_flag,
+                                                    p.status, p.wait_limit_ns));
+  if (ok) {
+    e.parity ^= 1u << i;
+    e.inflight &= ~(1u << i);
+  }
+  return ok;
+}
+
+// This warp's stores of a tile are complete (the caller waited for its bulk
+// groups): count it in the CTA's slot for that tile. The warp that completes
+// the count publishes the CTA's part of the tile with one release, so no
+// warp waits for another. Slot counters only grow; the tile's last arrival
+// is the one that makes the count a multiple of kEpiWarps. A slot is reused
+// four tiles later, after every warp has confirmed the tile that used it.
+__device__ __forceinline__ void confirm_tile(uint32_t* slot_count, int* done_cnt) {
+  static_assert((kEpiWarps & (kEpiWarps - 1)) == 0, "kEpiWarps must be a power of two");
+  fence_proxy_async_global();
+  if ((atom_add_acq_rel_cta(slot_count, 1u) & (kEpiWarps - 1)) == kEpiWarps - 1)
+    red_release_gpu_add(done_cnt, 1);
 }
 
 // Apply: x' = alpha x + beta D with x = hi + lo, for this lane's row.
@@ -437,6 +481,7 @@ __device__ __forceinline__ bool epi_reduce(const NsGemmParams& p, EpiRing& e, co
   constexpr int kAhead = kEpiBufs - 1;  // partials in flight beyond the one being summed
   if (lane == 0) {
     for (int s = 0; s < kAhead && s < ks; ++s) {
+      e.inflight |= 1u << s;
       mbar_arrive_expect_tx(&e.bar[s], kEpiChunkBytes);
       tma_load_2d(e.base + s * kEpiChunkBytes, pmap, &e.bar[s], pcol, prow0 + s * kTile);
     }
@@ -450,14 +495,16 @@ __device__ __forceinline__ bool epi_reduce(const NsGemmParams& p, EpiRing& e, co
     __syncwarp();
     if (lane == 0 && s + kAhead < ks) {
       const int slot = (s + kAhead) % kEpiBufs;
+      e.inflight |= 1u << slot;
       mbar_arrive_expect_tx(&e.bar[slot], kEpiChunkBytes);
       tma_load_2d(e.base + slot * kEpiChunkBytes, pmap, &e.bar[slot], pcol, prow0 + (s + kAhead) * kTile);
     }
     const int slot = s % kEpiBufs;
-    const bool ok = mbar_wait(&e.bar[slot], (e.parity >> slot) & 1u, abort_flag, p.status,
-                              p.wait_limit_ns);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&e.bar[slot], (e.parity >> slot) & 1u,
+                                                      abort_flag, p.status, p.wait_limit_ns));
+    if (!ok) return false;  // the load stays outstanding, to be drained
     e.parity ^= 1u << slot;
-    if (!__all_sync(0xffffffffu, ok)) return false;
+    e.inflight &= ~(1u << slot);
     const uint8_t* b = e.base + slot * kEpiChunkBytes;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
@@ -501,10 +548,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
-  uint64_t* pub = done + 1;     // per accumulator: this CTA's epilogue warps have stored the tile
-  uint64_t* epibar = pub + 2;   // kEpiWarps x kEpiBufs
+  uint64_t* epibar = done + 1;  // kEpiWarps x kEpiBufs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + kEpiWarps * kEpiBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* pubcnt = tmem_slot + 2;  // kPubSlots: epilogue warps that stored a tile, per slot
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -524,9 +571,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 2 * kEpiWarps);  // the leader's: both CTAs' epilogue warps
     }
     mbar_init(done, 1);
-    for (int a = 0; a < 2; ++a) mbar_init(&pub[a], kEpiWarps);
     for (int w = 0; w < kEpiWarps * kEpiBufs; ++w) mbar_init(&epibar[w], 1);
     *abort_flag = 0;
+    for (int i = 0; i < kPubSlots; ++i) pubcnt[i] = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -644,23 +691,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ---------------------------------------------------------------- epilogue
     // warp w may read TMEM lanes 32*(w%4)..+31 (this CTA's tile rows); warps
     // 2..5 take accumulator columns 0..127 and warps 6..9 columns 128..255.
+    //
+    // Loads run ahead across tiles: while this warp works through a tile's
+    // chunks, each freed buffer takes the load of the chunk kEpiBufs positions
+    // ahead, which near the end of the tile is one of the next tile's first
+    // chunks (issued only once the phase that tile reads is seen finished,
+    // checked without waiting). A tile is published one tile late: its
+    // stores complete while the next tile is worked on, and each warp
+    // confirms it after that tile's chunk loop. Before any wait on the next
+    // tile's dependency the pending tile is confirmed at once, so a pending
+    // publish never holds up a tile that needs it.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int ew = warp - 2;
-    EpiRing e{epibuf + ew * kEpiBufBytes, &epibar[ew * kEpiBufs], 0u, 0u};
+    const int irank = static_cast<int>(rank);
+    EpiRing e{epibuf + ew * kEpiBufBytes, &epibar[ew * kEpiBufs], 0u, 0u, 0u};
     const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
     constexpr int kChunks = 128 / kEpiCols;  // chunks per warp per tile
+    static_assert(kEpiBufs <= kChunks, "the loads of one tile fill the ring");
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = pair; ok && tile < ntiles; tile += npairs) {
-      const Tile T = decode_tile(p, tile);
+    int* pend_cnt = nullptr;   // lane 0: the tile whose publish is pending
+    uint32_t pend_slot = 0;
+    uint32_t seq = 0;          // MMA tiles handled by this warp
+    int t_issued = 0;          // lane 0: loads of the current tile already issued
+    int tile = pair;
+    Tile T;
+    if (tile < ntiles) T = decode_tile(p, tile);
+    while (ok && tile < ntiles) {
       const BankPlan& bp = p.bank[T.bank];
+      const int ntile = tile + npairs;
+      const bool has_next = ntile < ntiles;
+      Tile N;
+      if (has_next) N = decode_tile(p, ntile);
+      const bool next_loads = has_next && epi_has_loads(N);
+      int n_issued = 0;        // lane 0: loads of N issued during this tile
+      bool n_ready = false;    // lane 0: N's dependency seen finished
       if (T.phase == kReduce) {  // no accumulator: sum the split partials
-        if (lane == 0 && !wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit))
-          ok = false;
+        // the Reduce needs every ring buffer free and waits on its dependency
+        if (lane == 0) {
+          bulk_wait_all();
+          if (pend_cnt) {
+            confirm_tile(&pubcnt[pend_slot], pend_cnt);
+            pend_cnt = nullptr;
+          }
+          if (!wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) ok = false;
+        }
         if (!__all_sync(0xffffffffu, ok)) break;
-        if (!epi_reduce(p, e, T, bp, lane, static_cast<int>(rank), q, half, abort_flag)) {
+        if (!epi_reduce(p, e, T, bp, lane, irank, q, half, abort_flag)) {
           ok = false;
           break;
         }
@@ -670,28 +749,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           red_release_gpu_add(T.done_cnt, 1);
         }
         __syncwarp();
+        tile = ntile;
+        if (has_next) T = N;
+        t_issued = 0;
         continue;
       }
       const bool split = T.phase == kGram && bp.ksplit > 1;
       const int prow = (T.mat * bp.tiles_sym + T.sym_t) * bp.ksplit * kTile + T.split * kTile +
-                       kBM * static_cast<int>(rank) + 32 * q;
-      const int r0 = T.m0 + kBM * static_cast<int>(rank) + 32 * q;  // first row of this warp
-      const int cw = T.n0 + half * 128;                              // first column of this warp
-      const bool loads = T.phase != kGram;
-      // the epilogue's own TMA loads read the same finished phase as the MMAs;
-      // the first kEpiBufs chunks of the tile are requested now, while its
-      // MMAs run (each tile ends with all of its stores complete, so every
-      // buffer is free); a later chunk reuses a buffer once its store has
-      // read it
-      if (lane == 0 && loads) {
-        if (!wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) ok = false;
-        else
-          for (int j = 0; j < kChunks && j < kEpiBufs; ++j) epi_issue_load(p, e, T, bp, r0, cw + j * kEpiCols, e.chunk + j);
+                       kBM * irank + 32 * q;
+      const int r0 = T.m0 + kBM * irank + 32 * q;  // first row of this warp
+      const int cw = T.n0 + half * 128;            // first column of this warp
+      const bool loads = epi_has_loads(T);
+      if (lane == 0) {
+        // a pending publish must not hold up this tile: confirm it first
+        // whenever this tile's dependency is not yet met
+        if (pend_cnt && !dependency_met(T)) {
+          bulk_wait_all();
+          confirm_tile(&pubcnt[pend_slot], pend_cnt);
+          pend_cnt = nullptr;
+        }
+        if (loads) {
+          // the epilogue's own loads read the same finished phase as the MMAs
+          if (!wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) {
+            ok = false;
+          } else if (t_issued < kEpiBufs) {
+            bulk_wait_read<0>();  // the previous tile's buffers have been read out
+            for (int j = t_issued; j < kEpiBufs; ++j)
+              epi_issue_chunk(p, e, T, irank, q, half, j, e.chunk + j);
+          }
+        }
       }
       if (!__all_sync(0xffffffffu, ok)) break;
       // the tcgen05.ld below is warp-collective: leave only if the whole warp does
       const bool got = mbar_wait_cluster(&tfull[acc], acc_phase, abort_flag, p.status, limit);
-      if (!__all_sync(0xffffffffu, got)) break;
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                           static_cast<uint32_t>(acc * kBN + half * 128);
@@ -719,12 +813,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             epi_sym(T, bp, buf, lane, r);
           epi_store(p, T, bp, buf, r0, c0, lane);
         }
-        if (loads && j + kEpiBufs < kChunks) {
-          // chunk j's buffer takes chunk j + kEpiBufs once its store has read it
+        // buffer k % kEpiBufs next holds position k + kEpiBufs: a later chunk
+        // of this tile or one of the next tile's first chunks
+        const int ja = j + kEpiBufs;
+        if (ja < kChunks ? loads : next_loads) {
           __syncwarp();
           if (lane == 0) {
-            bulk_wait_read<0>();
-            epi_issue_load(p, e, T, bp, r0, c0 + kEpiBufs * kEpiCols, k + kEpiBufs);
+            if (ja < kChunks) {
+              bulk_wait_read<0>();
+              epi_issue_chunk(p, e, T, irank, q, half, ja, k + kEpiBufs);
+            } else if (n_issued == ja - kChunks && (n_ready || (n_ready = dependency_met(N)))) {
+              bulk_wait_read<0>();
+              fence_proxy_async_global();  // after the acquire, before the async-proxy reads
+              epi_issue_chunk(p, e, N, irank, q, half, n_issued, k + kEpiBufs);
+              ++n_issued;
+            }
           }
         }
         e.chunk = k + 1;
@@ -734,24 +837,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
-        // this warp's part of the tile is in global memory
-        bulk_wait_all();
-        fence_proxy_async_global();
-        mbar_arrive(&pub[acc]);
-        // the CTA's part is complete once every epilogue warp's is: the first
-        // epilogue warp publishes it (one release per CTA and tile)
-        if (ew == 0) {
-          if (mbar_wait(&pub[acc], acc_phase, abort_flag, p.status, limit))
-            red_release_gpu_add(T.done_cnt, 1);
-          else
-            ok = false;
+        // the previous tile's stores are the groups before this tile's kChunks
+        if (pend_cnt) {
+          bulk_wait<kChunks>();
+          confirm_tile(&pubcnt[pend_slot], pend_cnt);
         }
+        pend_cnt = T.done_cnt;
+        pend_slot = seq % kPubSlots;
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++seq;
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
+      tile = ntile;
+      if (has_next) T = N;
+      t_issued = n_issued;
     }
-    if (lane == 0) bulk_wait_all();  // every bulk store of this warp has completed
+    if (lane == 0) {
+      bulk_wait_all();  // every bulk store of this warp has completed
+      if (ok && pend_cnt) confirm_tile(&pubcnt[pend_slot], pend_cnt);
+      // after an error, loads issued ahead may still be in flight: let them
+      // land before the CTA's shared memory is released
+      for (int i = 0; i < kEpiBufs; ++i)
+        if (e.inflight & (1u << i)) drain_wait(&e.bar[i], (e.parity >> i) & 1u, limit);
+    }
     __syncwarp();
   }
 

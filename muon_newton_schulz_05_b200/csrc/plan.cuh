@@ -24,7 +24,13 @@ constexpr int kTile = 256;         // GEMM tile (rows and cols) computed by one 
 constexpr int kBM = 128;           // tile rows held by one CTA of the pair
 constexpr int kBN = 256;           // tile cols (UMMA N); each CTA loads kBN/2 of B
 constexpr int kBK = 64;            // K per pipeline stage (one 128-byte swizzle row)
-constexpr int kStages = 4;         // TMA -> MMA pipeline depth (3 measured slower)
+#ifndef MUON_STAGES
+#define MUON_STAGES 4
+#endif
+#ifndef MUON_EPI_BUFS
+#define MUON_EPI_BUFS 3
+#endif
+constexpr int kStages = MUON_STAGES;  // TMA -> MMA pipeline depth (3 measured slower)
 constexpr int kATileBytes = kBM * kBK * 2;
 constexpr int kBTileBytes = (kBN / 2) * kBK * 2;
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
@@ -33,7 +39,8 @@ constexpr int kEpiRows = 32;       // epilogue chunk: 32 rows x 32 columns per w
 constexpr int kEpiCols = 32;
 constexpr int kEpiHalfBytes = kEpiRows * kEpiCols * 2;      // one bf16 chunk
 constexpr int kEpiChunkBytes = 2 * kEpiHalfBytes;           // hi + lo (Apply)
-constexpr int kEpiBufs = 3;                                 // chunk buffers per warp
+constexpr int kEpiBufs = MUON_EPI_BUFS;                     // chunk buffers per warp
+constexpr int kPubSlots = 4;                                // per-CTA publish counters (tiles in flight)
 constexpr int kEpiBufBytes = kEpiBufs * kEpiChunkBytes;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 1024 + 512;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, then epilogue

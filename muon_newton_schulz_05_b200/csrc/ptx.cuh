@@ -110,6 +110,24 @@ __device__ __forceinline__ void bulk_wait_read() {
 // Wait until every committed bulk store of this thread is complete.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Wait until at most N of this thread's most recent committed bulk store
+// groups are incomplete (all older ones have written global memory).
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Shared-memory atomic add with acquire-release semantics at CTA scope;
+// returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_cta(uint32_t* ptr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(smem_u32(ptr)), "r"(v)
+               : "memory");
+  return old;
+}
+
 // Generic-proxy shared-memory writes of this thread become visible to the
 // async proxy (TMA) once this fence and a synchronisation have been passed.
 __device__ __forceinline__ void fence_proxy_async_smem() {
