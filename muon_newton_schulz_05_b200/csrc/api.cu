@@ -174,6 +174,12 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
     p.kc = (kg + p.ksplit - 1) / p.ksplit;
     if (p.ksplit > 1) p.ksplit = (kg + p.kc - 1) / p.kc;  // no empty split
     p.tiles_red = p.ksplit > 1 ? p.tiles_sym * kRedSub : 0;
+    p.fd_apply = make_fastdiv(p.tiles_apply);
+    p.fd_nbn = make_fastdiv(p.Cp / kTile);
+    p.fd_gram = make_fastdiv(p.tiles_sym * p.ksplit);
+    p.fd_ksplit = make_fastdiv(p.ksplit);
+    p.fd_red = make_fastdiv(p.tiles_red);
+    p.fd_sym = make_fastdiv(p.tiles_sym);
     const size_t it_bytes = static_cast<size_t>(p.count) * padded * 2;
     const size_t sq_bytes = static_cast<size_t>(p.count) * p.rp * p.rp * 2;
     const size_t o_hi0 = take(it_bytes), o_hi1 = take(it_bytes), o_lo = take(it_bytes);
@@ -337,6 +343,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
     sym += plans[b].count * plans[b].tiles_sym;
     app += plans[b].count * plans[b].tiles_apply;
   }
+  gp.fd_step = make_fastdiv(static_cast<uint32_t>(gram + red + sym + app));
   gp.gram_begin[nbanks] = gram;
   gp.red_begin[nbanks] = red;
   gp.sym_begin[nbanks] = sym;

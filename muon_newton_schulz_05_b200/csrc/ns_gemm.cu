@@ -33,6 +33,7 @@
 #include "plan.cuh"
 #include "ptx.cuh"
 
+
 namespace muon {
 
 struct Tile {
@@ -71,7 +72,7 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   Tile T;
   const int G = p.gram_begin[p.nbanks], Rd = p.red_begin[p.nbanks], S = p.sym_begin[p.nbanks];
   const int per_iter = tiles_per_step(p);
-  T.iter = tile / per_iter;
+  T.iter = fdiv(tile, p.fd_step);
   int r = tile - T.iter * per_iter;
   const int* begin;
   if (r < G) {
@@ -106,26 +107,27 @@ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int tile) {
   T.a_sym = T.b_sym = 0;
   T.a_tmap = T.b_tmap = 0;
   if (T.phase == kApply) {
-    T.mat = local / bp.tiles_apply;
+    T.mat = fdiv(local, bp.fd_apply);
     const int t = local - T.mat * bp.tiles_apply;
     const int nbn = bp.Cp / kTile;
-    T.m0 = (t / nbn) * kTile;
-    T.n0 = (t % nbn) * kTile;
+    const int mrow = fdiv(t, bp.fd_nbn);
+    T.m0 = mrow * kTile;
+    T.n0 = (t - mrow * nbn) * kTile;
   } else {
     int t;
     if (T.phase == kGram) {
       const int per = bp.tiles_sym * bp.ksplit;
-      T.mat = local / per;
+      T.mat = fdiv(local, bp.fd_gram);
       const int t2 = local - T.mat * per;
-      t = t2 / bp.ksplit;
+      t = fdiv(t2, bp.fd_ksplit);
       T.split = t2 - t * bp.ksplit;
     } else if (T.phase == kReduce) {
-      T.mat = local / bp.tiles_red;
+      T.mat = fdiv(local, bp.fd_red);
       const int t3 = local - T.mat * bp.tiles_red;
       t = t3 / kRedSub;
       T.sub = t3 - t * kRedSub;
     } else {
-      T.mat = local / bp.tiles_sym;
+      T.mat = fdiv(local, bp.fd_sym);
       t = local - T.mat * bp.tiles_sym;
     }
     T.sym_t = t;
@@ -255,10 +257,13 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_majo
 // ---------------------------------------------------------------- epilogues
 // Each epilogue warp owns 32 accumulator rows and 128 of the 256 columns and
 // works through them in 32 x 32 chunks. Global traffic goes through TMA only,
-// through kEpiBufs chunk buffers per warp: the bulk loads of the chunks' inputs
-// (Apply: hi and lo of the iterate; Poly: A) run kEpiBufs chunks ahead, across
-// tile boundaries, and the stores of earlier chunks drain while later ones
-// are computed. Halves use the 64-byte swizzle of the TMA box (16-byte group g of
+// through kEpiBufs chunk buffers per warp: the bulk loads of a tile's first
+// chunks (Apply: hi and lo of the iterate; Poly: A) are issued when the tile
+// starts, while its MMAs run, and the stores of earlier chunks drain while
+// later ones are computed. (Loading the next tile's first chunks while the
+// current one is still being worked on measured slower: those loads compete
+// with the operand loads the tensor cores are waiting for.) Halves use the
+// 64-byte swizzle of the TMA box (16-byte group g of
 // row r at r*64 + ((g ^ ((r >> 1) & 3)) * 16)), so a lane reading or writing
 // its own row touches 8 distinct bank groups per quarter warp.
 __device__ __forceinline__ uint32_t swz64_off(int r, int g) {
@@ -268,8 +273,7 @@ __device__ __forceinline__ uint32_t swz64_off(int r, int g) {
 // Ring positions: every chunk this warp handles takes the next position k;
 // position k uses buffer k % kEpiBufs and load barrier k % kEpiBufs. A load
 // for position k is issued once position k - kEpiBufs has had its store read
-// out of the buffer, so it may be issued up to kEpiBufs positions early, also
-// for the first chunks of the warp's next tile (loads run across tiles).
+// out of the buffer.
 struct EpiRing {
   uint8_t* base;     // kEpiBufs buffers of kEpiChunkBytes (two halves each)
   uint64_t* bar;     // kEpiBufs load barriers
@@ -692,15 +696,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // warp w may read TMEM lanes 32*(w%4)..+31 (this CTA's tile rows); warps
     // 2..5 take accumulator columns 0..127 and warps 6..9 columns 128..255.
     //
-    // Loads run ahead across tiles: while this warp works through a tile's
-    // chunks, each freed buffer takes the load of the chunk kEpiBufs positions
-    // ahead, which near the end of the tile is one of the next tile's first
-    // chunks (issued only once the phase that tile reads is seen finished,
-    // checked without waiting). A tile is published one tile late: its
-    // stores complete while the next tile is worked on, and each warp
-    // confirms it after that tile's chunk loop. Before any wait on the next
-    // tile's dependency the pending tile is confirmed at once, so a pending
-    // publish never holds up a tile that needs it.
+    // The accumulator is handed back to the MMA as soon as the last chunk's
+    // TMEM load has landed in registers. A tile is published one tile late:
+    // its stores complete while the next tile is worked on, and each warp
+    // confirms it after that tile's chunk loop. Before this warp could wait
+    // on a tile whose dependency is not yet met, the pending tile is
+    // confirmed at once, so a pending publish never holds up a tile that
+    // needs it (a CTA keeps a publish pending only while its next tile can
+    // run, and that tile finishes).
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int ew = warp - 2;
@@ -715,19 +718,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int* pend_cnt = nullptr;   // lane 0: the tile whose publish is pending
     uint32_t pend_slot = 0;
     uint32_t seq = 0;          // MMA tiles handled by this warp
-    int t_issued = 0;          // lane 0: loads of the current tile already issued
-    int tile = pair;
-    Tile T;
-    if (tile < ntiles) T = decode_tile(p, tile);
-    while (ok && tile < ntiles) {
+    for (int tile = pair; ok && tile < ntiles; tile += npairs) {
+      const Tile T = decode_tile(p, tile);
       const BankPlan& bp = p.bank[T.bank];
-      const int ntile = tile + npairs;
-      const bool has_next = ntile < ntiles;
-      Tile N;
-      if (has_next) N = decode_tile(p, ntile);
-      const bool next_loads = has_next && epi_has_loads(N);
-      int n_issued = 0;        // lane 0: loads of N issued during this tile
-      bool n_ready = false;    // lane 0: N's dependency seen finished
       if (T.phase == kReduce) {  // no accumulator: sum the split partials
         // the Reduce needs every ring buffer free and waits on its dependency
         if (lane == 0) {
@@ -749,9 +742,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           red_release_gpu_add(T.done_cnt, 1);
         }
         __syncwarp();
-        tile = ntile;
-        if (has_next) T = N;
-        t_issued = 0;
         continue;
       }
       const bool split = T.phase == kGram && bp.ksplit > 1;
@@ -761,21 +751,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int cw = T.n0 + half * 128;            // first column of this warp
       const bool loads = epi_has_loads(T);
       if (lane == 0) {
+        // one acquire of the dependency counter serves both checks below
+        const bool ready = !(pend_cnt || loads) || dependency_met(T);
         // a pending publish must not hold up this tile: confirm it first
         // whenever this tile's dependency is not yet met
-        if (pend_cnt && !dependency_met(T)) {
+        if (pend_cnt && !ready) {
           bulk_wait_all();
           confirm_tile(&pubcnt[pend_slot], pend_cnt);
           pend_cnt = nullptr;
         }
         if (loads) {
-          // the epilogue's own loads read the same finished phase as the MMAs
-          if (!wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) {
+          // the epilogue's own loads read the same finished phase as the MMAs;
+          // the first kEpiBufs chunks are requested now, while the MMAs run
+          if (!ready && !wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) {
             ok = false;
-          } else if (t_issued < kEpiBufs) {
+          } else {
+            fence_proxy_async_global();
             bulk_wait_read<0>();  // the previous tile's buffers have been read out
-            for (int j = t_issued; j < kEpiBufs; ++j)
-              epi_issue_chunk(p, e, T, irank, q, half, j, e.chunk + j);
+            for (int j = 0; j < kEpiBufs; ++j) epi_issue_chunk(p, e, T, irank, q, half, j, e.chunk + j);
           }
         }
       }
@@ -803,6 +796,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tmem_ld_wait();
+        if (j == kChunks - 1) {
+          // every accumulator column of this warp is in registers: hand the
+          // accumulator back. The arrive has the default (CTA-scope release)
+          // semantics: a cluster-scope release measured ~14 % of the
+          // epilogue's time per tile, and the TMEM reads it orders have
+          // completed (tcgen05.wait::ld) before it. Lane 1 arrives; lane 0
+          // issues the bulk stores.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 1) mbar_arrive_cluster_cta(tempty_leader + 8u * static_cast<uint32_t>(acc));
+        }
         uint8_t* buf = ring_buf(e, k);
         if (split) {
           epi_partial(p, T, buf, lane, prow, half * 128 + j * kEpiCols, r);
@@ -813,30 +817,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             epi_sym(T, bp, buf, lane, r);
           epi_store(p, T, bp, buf, r0, c0, lane);
         }
-        // buffer k % kEpiBufs next holds position k + kEpiBufs: a later chunk
-        // of this tile or one of the next tile's first chunks
-        const int ja = j + kEpiBufs;
-        if (ja < kChunks ? loads : next_loads) {
+        if (loads && j + kEpiBufs < kChunks) {
+          // chunk j's buffer takes chunk j + kEpiBufs once its store has read it
           __syncwarp();
           if (lane == 0) {
-            if (ja < kChunks) {
-              bulk_wait_read<0>();
-              epi_issue_chunk(p, e, T, irank, q, half, ja, k + kEpiBufs);
-            } else if (n_issued == ja - kChunks && (n_ready || (n_ready = dependency_met(N)))) {
-              bulk_wait_read<0>();
-              fence_proxy_async_global();  // after the acquire, before the async-proxy reads
-              epi_issue_chunk(p, e, N, irank, q, half, n_issued, k + kEpiBufs);
-              ++n_issued;
-            }
+            bulk_wait_read<0>();
+            epi_issue_chunk(p, e, T, irank, q, half, j + kEpiBufs, k + kEpiBufs);
           }
         }
         e.chunk = k + 1;
       }
       if (!ok) break;
-      tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
         // the previous tile's stores are the groups before this tile's kChunks
         if (pend_cnt) {
           bulk_wait<kChunks>();
@@ -848,15 +841,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       ++seq;
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
-      tile = ntile;
-      if (has_next) T = N;
-      t_issued = n_issued;
     }
     if (lane == 0) {
       bulk_wait_all();  // every bulk store of this warp has completed
       if (ok && pend_cnt) confirm_tile(&pubcnt[pend_slot], pend_cnt);
-      // after an error, loads issued ahead may still be in flight: let them
-      // land before the CTA's shared memory is released
+      // after an error, loads may still be in flight: let them land before
+      // the CTA's shared memory is released
       for (int i = 0; i < kEpiBufs; ++i)
         if (e.inflight & (1u << i)) drain_wait(&e.bar[i], (e.parity >> i) & 1u, limit);
     }

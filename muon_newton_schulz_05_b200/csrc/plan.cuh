@@ -48,6 +48,27 @@ constexpr int kChunk = 8192;       // padded elements per block in the momentum 
 constexpr int kMaxMaps = 14;
 
 enum Phase : int { kGram = 0, kPoly = 1, kApply = 2, kReduce = 3 };
+
+// Division by a divisor that is fixed for a launch, as a multiply and a shift
+// (division by invariant integers, Granlund and Montgomery): with
+// l = ceil(log2 d) and mul = floor(2^32 (2^l - d) / d) + 1,
+// n / d = (umulhi(n, mul) + n) >> l for 0 <= n < 2^31.
+struct FastDiv {
+  uint32_t mul, shift;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  if (d == 0) d = 1;  // unused divisors (a phase a bank does not have)
+  uint32_t l = 0;
+  while ((uint64_t(1) << l) < d) ++l;
+  const uint64_t mul = ((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1;
+  return FastDiv{static_cast<uint32_t>(mul), l};
+}
+
+__device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+  const uint32_t u = static_cast<uint32_t>(n);
+  return static_cast<int>((__umulhi(u, f.mul) + u) >> f.shift);
+}
 constexpr int kRedSub = 4;         // reduce sub-tiles per 256 x 256 tile (32 columns per warp)
 constexpr int kMaxSplit = 16;      // K splits of a Gram product
 
@@ -69,6 +90,9 @@ struct BankPlan {
   int ksplit;                   // K splits of the Gram product (1: none)
   int kc;                       // 64-deep K blocks per split
   int tiles_red;                // reduce sub-tiles (tiles_sym * kRedSub when split)
+  FastDiv fd_apply, fd_nbn;     // by tiles_apply, by Cp / 256
+  FastDiv fd_gram, fd_ksplit;   // by tiles_sym * ksplit, by ksplit
+  FastDiv fd_red, fd_sym;       // by tiles_red, by tiles_sym
   __nv_bfloat16* hi[2];         // iterate, high bf16 part (ping-pong)
   __nv_bfloat16* lo;            // iterate, low bf16 part (in place)
   __nv_bfloat16* A;             // Gram matrix, count x rp x rp; upper 256-blocks only
@@ -110,6 +134,7 @@ struct NsGemmParams {
   int apply_begin[MUON_MAX_BANKS + 1];  // prefix sums of count * tiles_apply
   int nbanks;
   int ns_steps;
+  FastDiv fd_step;                      // by the tiles of one Newton-Schulz step
   int keep_lo;                          // last step also stores lo (full-precision O)
   float coef[3 * MUON_MAX_NS_STEPS];    // (a, b, c) per step
   int* status;                          // device status word
