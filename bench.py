@@ -385,6 +385,7 @@ def run_native(args):
     value = job_throughput(world, K, total_ms)
 
     ns_avg_ms = statistics.mean(ns_ms)
+    step_ms = [ev[4 * s].elapsed_time(ev[4 * s + 3]) for s in range(K)]
     achieved = flops_step / (ns_avg_ms * 1e-3) / 1e12
     elem_bytes = sum(b.count * b.rows * b.cols for b in w.banks)
     # algorithmic bytes of the two elementwise passes per element:
@@ -478,12 +479,20 @@ def run_native(args):
         "roofline_square_1024x1024x64": square,
         "breakdown_ms": {"momentum_norm": statistics.mean(pre_ms), "ns_chain": ns_avg_ms,
                          "update": statistics.mean(post_ms)},
+        "step_ms_p10_p50_p90": _percentiles(step_ms), "ns_chain_ms_p10_p50_p90": _percentiles(ns_ms),
         "elementwise_gbs": {"momentum_norm": pre_gbs, "update": post_gbs, "peak": peaks["hbm"]},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": n_launch * K,
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _percentiles(xs):
+    """p10, p50, p90 of a list of per-step times (nearest rank)."""
+    ys = sorted(xs)
+    pick = lambda q: ys[min(len(ys) - 1, max(0, int(round(q * (len(ys) - 1)))))]
+    return [pick(0.1), pick(0.5), pick(0.9)]
 
 
 def _roofline(achieved, peaks, flops, launch_ms, traffic, traffic_src):

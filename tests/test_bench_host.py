@@ -51,3 +51,8 @@ def test_roofline_fraction_is_of_the_burst_peak():
     r = bench._roofline(800.0, peaks, 1.0e12, 1.25, None, "none")
     assert r["peak"] == 1600.0 and r["frac"] == 0.5
     assert r["frac_of_sustained"] == pytest.approx(800.0 / 1400.0)
+
+
+def test_percentiles_nearest_rank():
+    assert bench._percentiles([5.0, 1.0, 3.0, 2.0, 4.0]) == [1.0, 3.0, 5.0]
+    assert bench._percentiles([2.0]) == [2.0, 2.0, 2.0]
