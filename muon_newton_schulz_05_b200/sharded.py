@@ -62,13 +62,14 @@ class ShardPlan:
     @classmethod
     def build(cls, shapes: Sequence[Tuple[int, int, int]], world: int,
               buckets: Optional[Sequence[Sequence[int]]] = None) -> "ShardPlan":
-        """buckets: lists of bank indices (default: one bucket with all banks).
+        """buckets: lists of bank indices (default: one bucket per bank, so the
+        exchange of later banks overlaps the step of earlier ones).
         Owners are assigned bucket by bucket with the load carried over, so
         each bucket and the whole step are both close to balanced."""
         shapes = [tuple(int(v) for v in s) for s in shapes]
         if world < 1:
             raise ValueError("world size must be >= 1")
-        groups = [list(g) for g in buckets] if buckets is not None else [list(range(len(shapes)))]
+        groups = [list(g) for g in buckets] if buckets is not None else [[b] for b in range(len(shapes))]
         seen = sorted(b for g in groups for b in g)
         if seen != list(range(len(shapes))):
             raise ValueError("buckets must list every bank exactly once")
@@ -387,13 +388,18 @@ class ShardedBankMuon:
     buffer in place. Momenta (and the EMA) exist only for the owned matrices.
     A training loop may call `grad_ready(b)` as soon as bank b's gradients
     are final, then `finish(hp)`; `step(hp)` does both.
+    per_bank=False (default) steps every bank's owned matrices in one library
+    call (one Newton-Schulz chain over all of them: the most work per launch).
+    per_bank=True steps each bank as soon as its reduce-scatter has landed and
+    starts that bank's all-gather right after, so on NCCL the exchange of
+    later banks overlaps the chains of earlier ones.
     Requires rows * cols to be a multiple of 8, so that every matrix slot
     starts on a 16-byte boundary.
     """
 
     def __init__(self, shapes, param_dtype, grad_dtype, group=None, variant: str = "muon",
                  device=None, ema: bool = False, step_fn: Optional[Callable] = None,
-                 workspace_fn: Optional[Callable] = None):
+                 workspace_fn: Optional[Callable] = None, per_bank: bool = False):
         import torch
         import torch.distributed as dist
         if variant not in ("muon", "anvil"):
@@ -437,7 +443,9 @@ class ShardedBankMuon:
             self.momentum.append(state(True))
             self.momentum_slow.append(state(variant == "anvil"))
             self.ema.append(state(ema))
-        self.workspace = None
+        self.per_bank = bool(per_bank)
+        self.workspace = None                      # one call over all banks
+        self.workspaces: List = [None] * len(shapes)  # per_bank: one per bank
         self._ema_ready = False
         self._pending: List = [None] * len(shapes)
 
@@ -468,36 +476,68 @@ class ShardedBankMuon:
     def finish(self, hp) -> None:
         """Step the owned matrices of every bank (all must be grad_ready) with
         one library call, then all-gather every parameter buffer in place."""
-        from . import Bank
         if any(w is None for w in self._pending):
             raise RuntimeError("every bank needs grad_ready before finish")
-        for w in self._pending:
-            if w is not True:
-                w.wait()
-        banks = []
-        for b, (lo, hi) in enumerate(self.owned):
-            if hi == lo:
-                continue
-            p, g = self.params[b][lo:hi], self.grads[b][lo:hi]
-            if self.ema[b] is not None and not self._ema_ready:
-                self.ema[b].copy_(p)  # the average starts at the parameters it averages
-            banks.append(Bank(p, g, self.momentum[b], self.momentum_slow[b], self.ema[b]))
-        if banks:
-            if self.workspace is None:
-                self.workspace = self.workspace_fn([bk.shape for bk in banks])
-            self.step_fn(banks, hp, self.workspace)
+        nb = len(self.layout.banks)
         works = []
-        for b in range(len(self.layout.banks)):
-            flat, seg = self._pflat[b], self._segment(self._pflat[b], b)
-            if self.gloo:
-                self.dist.all_gather(list(flat.chunk(self.world)), seg.clone(), group=self.group)
-            else:
-                works.append(self.dist.all_gather_into_tensor(flat, seg, group=self.group,
-                                                              async_op=True))
+        if self.per_bank:
+            for b in range(nb):
+                self._wait_rs(b)
+                bank = self._owned_bank(b)
+                if bank is not None:
+                    if self.workspaces[b] is None:
+                        self.workspaces[b] = self.workspace_fn([bank.shape])
+                    self.step_fn([bank], hp, self.workspaces[b])
+                works.append(self._all_gather(b))
+        else:
+            for b in range(nb):
+                self._wait_rs(b)
+            banks = [bk for bk in (self._owned_bank(b) for b in range(nb)) if bk is not None]
+            if banks:
+                if self.workspace is None:
+                    self.workspace = self.workspace_fn([bk.shape for bk in banks])
+                self.step_fn(banks, hp, self.workspace)
+            works = [self._all_gather(b) for b in range(nb)]
         for w in works:
-            w.wait()
-        self._pending = [None] * len(self.layout.banks)
+            if w is not None:
+                w.wait()
+        self._pending = [None] * nb
         self._ema_ready = True
+
+    def _wait_rs(self, b: int) -> None:
+        if self._pending[b] is not True:
+            self._pending[b].wait()
+
+    def _owned_bank(self, b: int):
+        """The library's Bank for this rank's matrices of bank b (None if none)."""
+        from . import Bank
+        lo, hi = self.owned[b]
+        if hi == lo:
+            return None
+        p, g = self.params[b][lo:hi], self.grads[b][lo:hi]
+        if self.ema[b] is not None and not self._ema_ready:
+            self.ema[b].copy_(p)  # the average starts at the parameters it averages
+        return Bank(p, g, self.momentum[b], self.momentum_slow[b], self.ema[b])
+
+    def _all_gather(self, b: int):
+        """Start bank b's in-place all-gather: its work handle (None on gloo,
+        where it has completed)."""
+        flat, seg = self._pflat[b], self._segment(self._pflat[b], b)
+        if self.gloo:
+            self.dist.all_gather(list(flat.chunk(self.world)), seg.clone(), group=self.group)
+            return None
+        return self.dist.all_gather_into_tensor(flat, seg, group=self.group, async_op=True)
+
+    def device_status(self) -> int:
+        """Synchronises and returns the first non-zero device status of this
+        rank's workspaces (0 when all are clear)."""
+        from . import device_status
+        for ws in [self.workspace] + list(self.workspaces):
+            if ws is not None:
+                st = device_status(ws)
+                if st:
+                    return st
+        return 0
 
     def step(self, hp) -> None:
         for b in range(len(self.layout.banks)):

@@ -104,8 +104,9 @@ def test_sharded_single_rank_equals_direct_step_and_oracle(nccl_group, variant, 
             assert torch.equal(out[b], ema[b])
 
 
+@pytest.mark.parametrize("per_bank", [False, True])
 @pytest.mark.parametrize("variant", ["muon", "anvil"])
-def test_bank_storage_single_rank_equals_direct_step_and_oracle(nccl_group, variant):
+def test_bank_storage_single_rank_equals_direct_step_and_oracle(nccl_group, variant, per_bank):
     """ShardedBankMuon (owner-ordered bank storage, in-place reduce-scatter and
     all-gather) on one rank: bitwise a direct call of the library, and the
     oracle on the second step (fp32 parameters: O recovered from the step)."""
@@ -114,7 +115,7 @@ def test_bank_storage_single_rank_equals_direct_step_and_oracle(nccl_group, vari
     hp = _hparams(variant)
     ohp = hp_dict(hp)
     opt = ShardedBankMuon(SHAPES, torch.float32, torch.bfloat16, variant=variant, device=DEV,
-                          ema=(variant == "anvil"))
+                          ema=(variant == "anvil"), per_bank=per_bank)
     init = _bank(2, 0.02)
     for p, p0 in zip(opt.params, init):
         p.copy_(p0)
@@ -147,7 +148,7 @@ def test_bank_storage_single_rank_equals_direct_step_and_oracle(nccl_group, vari
                                      picks, "f32")
                 else:
                     check_muon_step(th0, opt.params[b], grads[b], m0, mom[b], ohp, picks, "f32")
-    assert mb.device_status(ws) == 0 and mb.device_status(opt.workspace) == 0
+    assert mb.device_status(ws) == 0 and opt.device_status() == 0
     if variant == "anvil":
         out = [torch.zeros(c, r, k, device=DEV) for c, r, k in SHAPES]
         opt.gather_ema(out)

@@ -300,10 +300,16 @@ def test_sharded_state_resumes_bitwise():
 
 def test_plan_owns_every_matrix_once_and_balances_gpt_bank():
     for world in (1, 2, 4, 8):
-        plan = ShardPlan.build(GPT_SHAPES, world)
-        for b, (count, rows, cols) in enumerate(GPT_SHAPES):
-            got = sorted(i for r in range(world) for i in plan.buckets[0].owned[r][b])
-            assert got == list(range(count))
+        for buckets in (None, [[0, 1, 2]]):   # default: one bucket per bank
+            plan = ShardPlan.build(GPT_SHAPES, world, buckets)
+            if buckets is None:
+                assert [bk.banks for bk in plan.buckets] == [[0], [1], [2]]
+            for b, (count, rows, cols) in enumerate(GPT_SHAPES):
+                k, j = next((k, j) for k, bk in enumerate(plan.buckets)
+                            for j, x in enumerate(bk.banks) if x == b)
+                got = sorted(i for r in range(world) for i in plan.buckets[k].owned[r][j])
+                assert got == list(range(count))
+        plan = ShardPlan.build(GPT_SHAPES, world, [[0, 1, 2]])
         total = sum(c * ns_work(r, k) for c, r, k in GPT_SHAPES)
         assert abs(sum(plan.load) - total) < 1e-6 * total
         # 72 matrices of two weights: greedy lands within one small matrix of even
@@ -342,7 +348,7 @@ def test_plan_rejects_bad_buckets():
 from muon_newton_schulz_05_b200.sharded import OwnerLayout  # noqa: E402
 
 
-def _bank_rank_main(rank, world, port, variant, steps, order, out):
+def _bank_rank_main(rank, world, port, variant, steps, order, out, per_bank=False):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     from muon_newton_schulz_05_b200.sharded import ShardedBankMuon
@@ -351,7 +357,7 @@ def _bank_rank_main(rank, world, port, variant, steps, order, out):
     try:
         opt = ShardedBankMuon(SHAPES, torch.bfloat16, torch.float32, variant=variant,
                               ema=(variant == "anvil"), step_fn=_oracle_step_fn(variant),
-                              workspace_fn=lambda shapes: None)
+                              workspace_fn=lambda shapes: None, per_bank=per_bank)
         for p, p0 in zip(opt.params, _params(SHAPES)):
             p.copy_(p0)
         hp = _hparams(variant)
@@ -373,9 +379,10 @@ def _bank_rank_main(rank, world, port, variant, steps, order, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("variant,world,order", [("muon", 2, [0, 1, 2]), ("anvil", 2, [2, 1, 0]),
-                                                 ("muon", 3, [1, 0, 2])])
-def test_bank_storage_step_equals_single_process_step(variant, world, order):
+@pytest.mark.parametrize("variant,world,order,per_bank",
+                         [("muon", 2, [0, 1, 2], False), ("anvil", 2, [2, 1, 0], True),
+                          ("muon", 3, [1, 0, 2], False), ("muon", 2, [1, 2, 0], True)])
+def test_bank_storage_step_equals_single_process_step(variant, world, order, per_bank):
     """Every rank ends with the bank one process gets by stepping every matrix
     on the mean of the ranks' gradients (gradients summed in the same order on
     both sides for two ranks; three ranks use integer-exact sums below)."""
@@ -383,8 +390,8 @@ def test_bank_storage_step_equals_single_process_step(variant, world, order):
     steps = 2
     with mp.Manager() as mgr:
         out = mgr.dict()
-        mp.spawn(_bank_rank_main, args=(world, port, variant, steps, order, out), nprocs=world,
-                 join=True)
+        mp.spawn(_bank_rank_main, args=(world, port, variant, steps, order, out, per_bank),
+                 nprocs=world, join=True)
         res = dict(out)
     # every matrix owned by exactly one rank
     for b, (count, _, _) in enumerate(SHAPES):
