@@ -46,9 +46,9 @@ SQUARE_ID = 3
 # sources change the figure no longer describes the kernel and is reported
 # as null.
 NS_CHAIN_TRAFFIC = {
-    2: {"bytes": 5.190445e9, "source_sha16": "4270d9457ccba00b",
+    2: {"bytes": 5.190445e9, "source_sha16": "db8a86ce544f4f8c",
         "capture": "ncu --set full, one chain launch of the GPT-124M bank (second step)"},
-    3: {"bytes": 4.875267e9, "source_sha16": "4270d9457ccba00b",
+    3: {"bytes": 4.875267e9, "source_sha16": "db8a86ce544f4f8c",
         "capture": "ncu --set full, one chain launch of the 64 x 1024^2 bank (second step)"},
 }
 KERNEL_SOURCES = ("ns_gemm.cu", "plan.cuh", "ptx.cuh")
@@ -88,13 +88,23 @@ def _peaks():
         return dict(hbm=6650.0, burst=1590.0, sustained=1400.0, src="fallback")
 
 
+def code_only(text: str) -> str:
+    """C/CUDA source without comments, trailing blanks and empty lines, so
+    that editing a comment does not change what a hash of it describes."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
 def kernel_source_sha16() -> str:
-    """Hash of the Newton-Schulz kernel's sources (what a traffic figure describes)."""
+    """Hash of the Newton-Schulz kernel's sources, code only (what a traffic
+    figure describes)."""
     import hashlib
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "muon_newton_schulz_05_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "muon_newton_schulz_05_b200", "csrc", f)) as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -25,7 +25,9 @@
 //   warps 2..9 epilogue: tcgen05.ld this CTA's 128 accumulator rows (warp w
 //              reads TMEM lanes 32*(w%4)..+31; two warps per lane quadrant
 //              split the 256 columns), apply the phase's axpy and store;
-//              one thread per CTA publishes the finished tile
+//              the accumulator goes back to the MMA as soon as its last
+//              columns are in registers, and the CTA's part of a tile is
+//              published one tile later by the last warp to confirm it
 // The epilogue of tile t overlaps the MMAs of tile t+1 through the two
 // accumulators. Every wait is bounded (muon::mbar_wait*).
 #include <cuda_runtime.h>

@@ -117,11 +117,12 @@ struct UpdBank {
 // are listed step by step, phase by phase (Gram, Reduce, Poly, Apply), bank by
 // bank, matrix by matrix; CTA pairs take them round-robin. A tile waits on
 // per-matrix counters for the phase it reads. When all eight epilogue warps
-// of a CTA have stored their part of an MMA tile, one thread of the CTA adds
-// 1 to the tile's phase counter (kTileParts per tile); a Reduce sub-tile is
-// published by every epilogue warp of both CTAs (kRedParts). Banks whose Gram K is much longer than the matrix is
-// wide split that product along K: the split tiles store fp32 partials and
-// Reduce sub-tiles sum them into A.
+// of a CTA have stored their part of an MMA tile (each confirms it after its
+// next tile's chunks, or at once when that tile would wait), the last of them
+// adds 1 to the tile's phase counter (kTileParts per tile); a Reduce sub-tile
+// is published by every epilogue warp of both CTAs (kRedParts). Banks whose
+// Gram K is much longer than the matrix is wide split that product along K:
+// the split tiles store fp32 partials and Reduce sub-tiles sum them into A.
 constexpr int kTileParts = 2;                // MMA tiles: one part per CTA of the pair
 constexpr int kRedParts = 2 * kEpiWarps;     // Reduce sub-tiles: one per epilogue warp of both CTAs
 

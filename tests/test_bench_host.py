@@ -56,3 +56,11 @@ def test_roofline_fraction_is_of_the_burst_peak():
 def test_percentiles_nearest_rank():
     assert bench._percentiles([5.0, 1.0, 3.0, 2.0, 4.0]) == [1.0, 3.0, 5.0]
     assert bench._percentiles([2.0]) == [2.0, 2.0, 2.0]
+
+
+def test_source_hash_ignores_comments():
+    a = "int f(int x) {  // doubles\n  return 2 * x; /* twice */\n}\n"
+    b = "// a header comment\nint f(int x) {\n\n  return 2 * x;\n}\n"
+    assert bench.code_only(a) == bench.code_only(b)
+    assert bench.code_only(a) != bench.code_only(a.replace("2 * x", "3 * x"))
+    assert bench.chain_traffic(2)[0] is not None   # the stored capture describes these sources
