@@ -632,23 +632,62 @@ def run_sharded(args):
         local_ms = l0.elapsed_time(l1) / K
     local_max = max_over_ranks(local_ms, dist, dev)
 
-    # end to end: this rank's gradients in from pinned host memory and the
-    # updated bank out, every step, on the step's stream
-    host_params = [torch.empty(p.shape, dtype=p.dtype).pin_memory() for p in opt.params]
+    # end to end: every step this rank's gradients come in from pinned host
+    # memory and the updated bank goes out, pipelined as a training loop would:
+    # the next step's gradients upload into a staging buffer on one copy
+    # stream while this step runs (a device copy moves them into the
+    # optimizer's gradient storage at the step's start), and a device snapshot
+    # of the parameters is read back on another copy stream during the next step
+    host_params = [[torch.empty(p.shape, dtype=p.dtype).pin_memory() for p in opt.params]
+                   for _ in range(2)]
+    stage = [[torch.empty_like(g) for g in opt.grads] for _ in range(2)]
+    snaps = [[torch.empty_like(p) for p in opt.params] for _ in range(2)]
+    up_s, down_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    up_done = [torch.cuda.Event() for _ in range(2)]
+    staged_free = [torch.cuda.Event() for _ in range(2)]
+    snap_done = [torch.cuda.Event() for _ in range(2)]
+    down_done = [torch.cuda.Event() for _ in range(2)]
     E = args.e2e_steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(E):
-        for g, hg in zip(opt.grads, host_grads):
-            g.copy_(hg, non_blocking=True)
+
+    def upload(i):
+        up_s.wait_event(staged_free[i])       # the step that read staging buffer i has started
+        with torch.cuda.stream(up_s):
+            for sg, hg in zip(stage[i], host_grads):
+                sg.copy_(hg, non_blocking=True)
+        up_done[i].record(up_s)
+
+    for i in range(2):
+        staged_free[i].record(stream)
+    upload(0)
+    for s_ in range(E):
+        i = s_ % 2
+        if s_ + 1 < E:
+            upload(1 - i)                      # the next step's gradients, during this step
+        stream.wait_event(up_done[i])
+        for g, sg in zip(opt.grads, stage[i]):
+            g.copy_(sg, non_blocking=True)
+        staged_free[i].record(stream)
         opt.step(H)
-        for hp_, p in zip(host_params, opt.params):
-            hp_.copy_(p, non_blocking=True)
+        if s_ >= 2:
+            stream.wait_event(down_done[i])    # snapshot i has been read back
+        for sn, p in zip(snaps[i], opt.params):
+            sn.copy_(p, non_blocking=True)
+        snap_done[i].record(stream)
+        down_s.wait_event(snap_done[i])
+        with torch.cuda.stream(down_s):
+            for hp_, sn in zip(host_params[i], snaps[i]):
+                hp_.copy_(sn, non_blocking=True)
+        down_done[i].record(down_s)
+    for i in range(min(E, 2)):
+        stream.wait_event(down_done[(E - 1 - i) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    host_params = host_params[0]
     h2d = sum(g.numel() * g.element_size() for g in host_grads)
     d2h = sum(p.numel() * p.element_size() for p in host_params)
     assert opt.workspace is None or mb.device_status(opt.workspace) == 0
@@ -680,7 +719,8 @@ def run_sharded(args):
         "e2e": {"value": E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "what": "per step and rank: pinned host->device copy of the rank's gradients, "
-                        "the sharded step, device->host copy of the updated bank"},
+                        "the sharded step, device->host copy of the updated bank; copies of "
+                        "neighbouring steps overlap the step on two copy streams"},
         "gpu_launches": launches_per_step(w) * K,
         "clocks": clk,
     }
