@@ -40,7 +40,7 @@ STATUS_NAMES = {
 EXPORTED = ("muon_abi_version", "muon_status_string", "muon_workspace_size", "muon_step",
             "anvil_step", "muon_orthogonalize", "ema_update", "readout_blend",
             "muon_device_status", "muon_set_debug", "muon_set_ns_events",
-            "muon_orthogonalize_static")
+            "muon_orthogonalize_static", "muon_chain_plan")
 
 
 class MuonError(RuntimeError):
@@ -80,6 +80,7 @@ _sig = {
     "muon_device_status": (_i32, [_vp, _sz, _vp, _i32]),
     "muon_set_debug": (_i32, [_i32, ctypes.c_double]),
     "muon_set_ns_events": (_i32, [_vp, _vp]),
+    "muon_chain_plan": (_i64, [ctypes.POINTER(_i64), _i32, _i32, ctypes.POINTER(_i32), _i64]),
     "muon_orthogonalize_static": (_i32, [_vp, _i32, _vp, _i32, _i64, _i64, _i64,
                                          ctypes.POINTER(CHparams), _vp]),
 }

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmuonb200.so")
 LIB_CHECK = os.path.join(PKG, "libmuonb200_check.so")
 SOURCES = ["api.cu", "elementwise.cu", "ns_gemm.cu"]
-HEADERS = ["plan.cuh", "ptx.cuh", "update_math.cuh", "check.cuh"]
+HEADERS = ["plan.cuh", "ptx.cuh", "tiles.cuh", "update_math.cuh", "check.cuh"]
 
 
 def nvcc() -> str:

@@ -11,6 +11,7 @@
 
 #include "muon_b200.h"
 #include "plan.cuh"
+#include "tiles.cuh"
 
 using namespace muon;
 
@@ -137,7 +138,8 @@ struct Shape3 {
   int64_t count, rows, cols;
 };
 
-// Fills plans (if base != nullptr) and returns the workspace bytes needed.
+// Returns the workspace bytes needed; fills plans if given (with the buffer
+// addresses inside the workspace at base, if base is given).
 size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan* plans) {
   size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
@@ -190,7 +192,11 @@ size_t plan_workspace(const Shape3* shapes, int nbanks, uint8_t* base, BankPlan*
     const size_t o_gpart = p.ksplit > 1 ? take(static_cast<size_t>(p.count) * p.tiles_sym * p.ksplit *
                                               kTile * kTile * 4)
                                        : 0;
-    if (base) {
+    if (plans) {
+      if (!base) {  // geometry only
+        plans[b] = p;
+        continue;
+      }
       p.hi[0] = reinterpret_cast<__nv_bfloat16*>(base + o_hi0);
       p.hi[1] = reinterpret_cast<__nv_bfloat16*>(base + o_hi1);
       p.lo = reinterpret_cast<__nv_bfloat16*>(base + o_lo);
@@ -268,6 +274,29 @@ UpdBank update_io(const muon_bank& b, const muon_hparams* hp) {
   return UpdBank{b.param, b.param_dtype, b.momentum_slow, b.ema, static_cast<float>(double(hp->lr) * s)};
 }
 
+// Tile prefix sums of the chain (list order: step, phase Gram / Reduce / Poly
+// / Apply, bank, matrix).
+void plan_chain(NsGemmParams& gp, const BankPlan* plans, int nbanks) {
+  gp.nbanks = nbanks;
+  int gram = 0, red = 0, sym = 0, app = 0;
+  for (int b = 0; b < nbanks; ++b) {
+    gp.bank[b] = plans[b];
+    gp.gram_begin[b] = gram;
+    gp.red_begin[b] = red;
+    gp.sym_begin[b] = sym;
+    gp.apply_begin[b] = app;
+    gram += plans[b].count * plans[b].tiles_sym * plans[b].ksplit;
+    red += plans[b].count * plans[b].tiles_red;
+    sym += plans[b].count * plans[b].tiles_sym;
+    app += plans[b].count * plans[b].tiles_apply;
+  }
+  gp.fd_step = make_fastdiv(static_cast<uint32_t>(gram + red + sym + app));
+  gp.gram_begin[nbanks] = gram;
+  gp.red_begin[nbanks] = red;
+  gp.sym_begin[nbanks] = sym;
+  gp.apply_begin[nbanks] = app;
+}
+
 muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_hparams* hp,
                      void* ws, size_t ws_bytes, cudaStream_t stream, const OrthoIO* oio) {
   int sms = 0, max_pairs = 0;
@@ -316,12 +345,10 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   if (launch_momentum_norm(mp, blocks, mats, stream) != cudaSuccess) return MUON_ERR_CUDA;
 
   // ---- Newton-Schulz chain
-  gp.nbanks = nbanks;
   gp.status = status;
   const double lim = g_debug.wait_limit_s > 0 ? g_debug.wait_limit_s : 2.0;
   gp.wait_limit_ns = static_cast<unsigned long long>(lim * 1e9);
   gp.fault = g_debug.fault;
-  for (int b = 0; b < nbanks; ++b) gp.bank[b] = plans[b];
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -332,22 +359,7 @@ muon_status run_step(Variant v, const muon_bank* banks, int nbanks, const muon_h
   gp.ns_steps = hp->ns_steps;
   gp.keep_lo = v == Variant::kOrtho ? 1 : 0;
   for (int i = 0; i < 3 * hp->ns_steps; ++i) gp.coef[i] = hp->coeffs[i];
-  int gram = 0, red = 0, sym = 0, app = 0;
-  for (int b = 0; b < nbanks; ++b) {
-    gp.gram_begin[b] = gram;
-    gp.red_begin[b] = red;
-    gp.sym_begin[b] = sym;
-    gp.apply_begin[b] = app;
-    gram += plans[b].count * plans[b].tiles_sym * plans[b].ksplit;
-    red += plans[b].count * plans[b].tiles_red;
-    sym += plans[b].count * plans[b].tiles_sym;
-    app += plans[b].count * plans[b].tiles_apply;
-  }
-  gp.fd_step = make_fastdiv(static_cast<uint32_t>(gram + red + sym + app));
-  gp.gram_begin[nbanks] = gram;
-  gp.red_begin[nbanks] = red;
-  gp.sym_begin[nbanks] = sym;
-  gp.apply_begin[nbanks] = app;
+  plan_chain(gp, plans, nbanks);
   if (launch_ns_gemm(gp, max_pairs, stream) != cudaSuccess) return MUON_ERR_CUDA;
   if (ev_after && cudaEventRecord(ev_after, stream) != cudaSuccess) return MUON_ERR_CUDA;
 
@@ -588,6 +600,34 @@ muon_status muon_set_ns_events(void* before_ns, void* after_ns) {
   g_ev_before = static_cast<cudaEvent_t>(before_ns);
   g_ev_after = static_cast<cudaEvent_t>(after_ns);
   return MUON_OK;
+}
+
+int64_t muon_chain_plan(const int64_t* shapes, int32_t nbanks, int32_t ns_steps, int32_t* tiles,
+                        int64_t tiles_cap) {
+  if (!shapes) return -static_cast<int64_t>(MUON_ERR_NULL);
+  if (nbanks < 1 || nbanks > MUON_MAX_BANKS) return -static_cast<int64_t>(MUON_ERR_SHAPE);
+  if (ns_steps < 1 || ns_steps > MUON_MAX_NS_STEPS) return -static_cast<int64_t>(MUON_ERR_HPARAM);
+  Shape3 sh[MUON_MAX_BANKS];
+  for (int b = 0; b < nbanks; ++b) {
+    sh[b] = {shapes[3 * b], shapes[3 * b + 1], shapes[3 * b + 2]};
+    const muon_status st = check_shape(sh[b].count, sh[b].rows, sh[b].cols);
+    if (st != MUON_OK) return -static_cast<int64_t>(st);
+  }
+  static thread_local NsGemmParams gp;  // large; kept off the stack
+  std::memset(&gp, 0, sizeof(gp));
+  BankPlan plans[MUON_MAX_BANKS];
+  plan_workspace(sh, nbanks, nullptr, plans);
+  plan_chain(gp, plans, nbanks);
+  gp.ns_steps = ns_steps;
+  const int64_t nt = static_cast<int64_t>(ns_steps) * tiles_per_step(gp);
+  if (tiles && tiles_cap >= 12 * nt)
+    for (int64_t t = 0; t < nt; ++t) {
+      const Tile T = decode_tile(gp, static_cast<int>(t));
+      int32_t* o = tiles + 12 * t;
+      o[0] = T.iter; o[1] = T.phase; o[2] = T.bank; o[3] = T.mat; o[4] = T.m0; o[5] = T.n0;
+      o[6] = T.kb0; o[7] = T.nkb; o[8] = T.a_map; o[9] = T.a_base; o[10] = T.b_map; o[11] = T.b_base;
+    }
+  return nt;
 }
 
 muon_status muon_set_debug(int32_t fault_mode, double wait_limit_seconds) {

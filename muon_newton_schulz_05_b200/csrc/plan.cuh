@@ -65,9 +65,14 @@ inline FastDiv make_fastdiv(uint32_t d) {
   return FastDiv{static_cast<uint32_t>(mul), l};
 }
 
-__device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+__host__ __device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
   const uint32_t u = static_cast<uint32_t>(n);
-  return static_cast<int>((__umulhi(u, f.mul) + u) >> f.shift);
+#ifdef __CUDA_ARCH__
+  const uint32_t hi = __umulhi(u, f.mul);
+#else
+  const uint32_t hi = static_cast<uint32_t>((static_cast<uint64_t>(u) * f.mul) >> 32);
+#endif
+  return static_cast<int>((hi + u) >> f.shift);
 }
 constexpr int kRedSub = 4;         // reduce sub-tiles per 256 x 256 tile (32 columns per warp)
 constexpr int kMaxSplit = 16;      // K splits of a Gram product
@@ -142,6 +147,11 @@ struct NsGemmParams {
   unsigned long long wait_limit_ns;
   int fault;                            // test hook (muon_set_debug)
 };
+
+__host__ __device__ __forceinline__ int tiles_per_step(const NsGemmParams& p) {
+  return p.gram_begin[p.nbanks] + p.red_begin[p.nbanks] + p.sym_begin[p.nbanks] +
+         p.apply_begin[p.nbanks];
+}
 
 // ---------------------------------------------------------- momentum + norm
 struct MomBank {
