@@ -208,11 +208,12 @@ muon_status muon_set_ns_events(void* before_ns, void* after_ns);
  * the given shapes (shapes[3b..3b+2] = count, rows, cols of bank b) and
  * ns_steps, as the kernel decodes it. Tiles are listed step by step, phase by
  * phase (Gram, Reduce, Poly, Apply), bank by bank, matrix by matrix. If
- * tiles_cap >= 12 * (number of tiles), tiles[12t..12t+11] = (step, phase
+ * tiles_cap >= 13 * (number of tiles), tiles[13t..13t+12] = (step, phase
  * (0 Gram, 1 Poly, 2 Apply, 3 Reduce), bank, matrix, first output row, first
  * output column, first 64-deep K block, K blocks, left operand map slot, left
- * operand base row, right operand map slot, right operand base row) of tile
- * t. Returns the number of tiles, or minus a muon_status on invalid input. */
+ * operand base row, right operand map slot, right operand base row, 1 if the
+ * right operand is the left one and is not loaded) of tile t. Returns the
+ * number of tiles, or minus a muon_status on invalid input. */
 int64_t muon_chain_plan(const int64_t* shapes, int32_t nbanks, int32_t ns_steps, int32_t* tiles,
                         int64_t tiles_cap);
 

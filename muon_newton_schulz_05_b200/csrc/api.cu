@@ -620,12 +620,13 @@ int64_t muon_chain_plan(const int64_t* shapes, int32_t nbanks, int32_t ns_steps,
   plan_chain(gp, plans, nbanks);
   gp.ns_steps = ns_steps;
   const int64_t nt = static_cast<int64_t>(ns_steps) * tiles_per_step(gp);
-  if (tiles && tiles_cap >= 12 * nt)
+  if (tiles && tiles_cap >= 13 * nt)
     for (int64_t t = 0; t < nt; ++t) {
       const Tile T = decode_tile(gp, static_cast<int>(t));
-      int32_t* o = tiles + 12 * t;
+      int32_t* o = tiles + 13 * t;
       o[0] = T.iter; o[1] = T.phase; o[2] = T.bank; o[3] = T.mat; o[4] = T.m0; o[5] = T.n0;
       o[6] = T.kb0; o[7] = T.nkb; o[8] = T.a_map; o[9] = T.a_base; o[10] = T.b_map; o[11] = T.b_base;
+      o[12] = T.same_ab;
     }
   return nt;
 }

@@ -464,14 +464,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (!withhold) {
             uint8_t* st = tiles + stage * kStageBytes;
             const uint32_t bar = full_leader + 8u * static_cast<uint32_t>(stage);
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+            // a diagonal block's right operand is the left one: not loaded
+            if (rank == 0)
+              mbar_arrive_expect_tx(&full[stage], T.same_ab ? 2 * kATileBytes : 2 * kStageBytes);
             const int k0 = (T.kb0 + kb) * kBK;
             const bool at = below_diagonal(T.a_sym, T.m0, k0);
             const bool bt = below_diagonal(T.b_sym, T.n0, k0);
             load_operand(st, at ? &p.maps[T.bank][T.a_tmap] : amap, bar, at ? 1 : T.a_mn, T.a_base,
                          T.m0 + kBM * rank, k0);
-            load_operand(st + kATileBytes, bt ? &p.maps[T.bank][T.b_tmap] : bmap, bar, bt ? 1 : T.b_mn,
-                         T.b_base, T.n0 + (kBN / 2) * rank, k0);
+            if (!T.same_ab)
+              load_operand(st + kATileBytes, bt ? &p.maps[T.bank][T.b_tmap] : bmap, bar, bt ? 1 : T.b_mn,
+                           T.b_base, T.n0 + (kBN / 2) * rank, k0);
             issued_parity[stage] = static_cast<int>(phase);
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -507,7 +510,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             }
             tc_fence_after();
             const uint32_t a_addr = smem_u32(tiles + stage * kStageBytes);
-            const uint32_t b_addr = a_addr + kATileBytes;
+            // on a diagonal block each CTA's half of the right operand (N rows
+            // 128 * rank ..) is its own rows of the left operand
+            const uint32_t b_addr = T.same_ab ? a_addr : a_addr + kATileBytes;
             // the producer's choice of orientation for this K block
             const int k0 = (T.kb0 + kb) * kBK;
             const int a_mn = below_diagonal(T.a_sym, T.m0, k0) ? 1 : T.a_mn;

@@ -16,6 +16,8 @@ struct Tile {
   int b_map, b_mn, b_base;
   int a_sym, b_sym;           // operand is A or B: blocks below the diagonal read transposed
   int a_tmap, b_tmap;         // the MN-major map for those blocks
+  int same_ab;                // diagonal block of a symmetric product: each CTA's half of
+                              // the right operand is its own rows of the left operand
   int* done_cnt;              // counter this tile's epilogue advances
   const int* dep_cnt;         // counter of the phase this tile reads
   int dep_target;             // value dep_cnt must reach first (0: nothing to wait for)
@@ -72,6 +74,7 @@ __host__ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int 
   T.sym_t = 0;
   T.a_sym = T.b_sym = 0;
   T.a_tmap = T.b_tmap = 0;
+  T.same_ab = 0;
   if (T.phase == kApply) {
     T.mat = fdiv(local, bp.fd_apply);
     const int t = local - T.mat * bp.tiles_apply;
@@ -101,6 +104,10 @@ __host__ __device__ __forceinline__ Tile decode_tile(const NsGemmParams& p, int 
     sym_tile(t, bp.rp / kTile, i, j);
     T.m0 = i * kTile;
     T.n0 = j * kTile;
+    // Gram and Poly read the same matrix on both sides (X X^T, A A); on a
+    // diagonal block both sides are the same 256 rows, in the same
+    // orientation for every K block
+    T.same_ab = (T.phase != kReduce && i == j) ? 1 : 0;
   }
   // Gram(k) reads X_k (all of Apply(k-1)); Reduce(k) sums all of Gram(k)'s
   // partials; Poly(k) reads A (all of Reduce(k), or of Gram(k) when the bank

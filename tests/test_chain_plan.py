@@ -33,9 +33,9 @@ def chain_plan(shapes, ns_steps):
     sh = (ctypes.c_int64 * (3 * len(shapes)))(*[v for s in shapes for v in s])
     nt = f(sh, len(shapes), ns_steps, None, 0)
     assert nt > 0, nt
-    til = np.zeros(12 * nt, dtype=np.int32)
+    til = np.zeros(13 * nt, dtype=np.int32)
     assert f(sh, len(shapes), ns_steps, til.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), til.size) == nt
-    return til.reshape(-1, 12)
+    return til.reshape(-1, 13)
 
 
 def pad(n):
@@ -145,6 +145,20 @@ def test_each_tile_reads_the_operands_of_its_product(name):
             assert (a_map, a_base, b_map, b_base) == (HI_K[cur], xbase, B_K, sbase)
         else:             # X <- aX + B X
             assert (a_map, a_base, b_map, b_base) == (B_K, sbase, HI_MN[cur], xbase)
+
+
+@pytest.mark.parametrize("name", sorted(SHAPES))
+def test_only_diagonal_symmetric_blocks_reuse_the_left_operand(name):
+    """The right operand is skipped exactly on the diagonal blocks of Gram and
+    Poly, where both sides are the same rows of the same matrix read the same
+    way (same map, same base row, same first row)."""
+    til = chain_plan(SHAPES[name], 2)
+    for t in til:
+        ph, m0, n0, same = t[1], t[4], t[5], t[12]
+        want = int(ph in (GRAM, POLY) and m0 == n0)
+        assert same == want, t
+        if same:
+            assert (t[8], t[9]) == (t[10], t[11])
 
 
 def test_invalid_plans_are_refused():
