@@ -40,6 +40,8 @@ def orth_gpu(x, coeffs, out_dtype=torch.float32, eps=1e-7):
 
 # ----------------------------------------------------------- orthogonalisation
 SHAPES = [(1, 256, 256), (1, 256, 512), (1, 512, 256), (2, 7, 13), (2, 13, 7), (1, 1, 1),
+          # a single row or column: X X^T is the squared norm, the result x / ||x|| * p(1)
+          (1, 1, 777), (1, 777, 1),
           (1, 129, 257), (1, 257, 129), (2, 384, 640), (1, 768, 3072), (1, 3072, 768),
           # Gram K much longer than the Gram is wide: the product is split along K
           (1, 256, 8192), (1, 8192, 256), (1, 300, 20000)]
