@@ -66,7 +66,9 @@ def _args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=40)
+    # the end-to-end leg: long enough that its first upload and last read-back,
+    # which nothing overlaps, weigh little against the steady state
+    ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-square", action="store_true",
                     help="skip the 64 x 1024^2 roofline line")
