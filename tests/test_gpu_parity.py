@@ -73,6 +73,25 @@ def test_orthogonalize_matches_oracle(shape, cname):
         assert sv_maxdiff(got, ref) <= sv_tol
 
 
+@pytest.mark.parametrize("rank", [1, 64])
+@pytest.mark.parametrize("shape", [(768, 768), (768, 3072), (3072, 768)])
+def test_orthogonalize_low_rank_gradients(rank, shape):
+    """Gradients of low rank (x^T dy over `rank` rows, as one small batch
+    gives): in their null space only the a X term acts, so the iterate's
+    rounding noise grows by a per step unless X is carried to more than bf16
+    precision through every step."""
+    R, C = shape
+    g = torch.Generator().manual_seed(rank * 7 + R)
+    x = torch.randn(rank, R, generator=g, dtype=torch.float64)
+    dy = torch.randn(rank, C, generator=g, dtype=torch.float64)
+    u = (x.T @ dy).to(torch.bfloat16)[None]
+    for coeffs in ([QUINTIC] * 5, [QUINTIC] * 6):
+        out = orth_gpu(u.to(DEV), coeffs).cpu()
+        ref = oracle.orthogonalize(f64(u[0]), coeffs, 1e-7)
+        assert rel_fro(f64(out[0]), ref) <= TOL_UPDATE, (len(coeffs), rel_fro(f64(out[0]), ref))
+        assert sv_maxdiff(f64(out[0]), ref) <= TOL_SV
+
+
 def test_orthogonalize_bf16_output_and_fp32_input():
     x = mi.spiked_gaussian(768, 768, 5, 1e-3, 4, 10.0)[None].to(DEV)
     out = orth_gpu(x, [QUINTIC] * 5, out_dtype=torch.bfloat16)
