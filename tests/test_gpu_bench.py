@@ -12,6 +12,7 @@ import os
 import socket
 import subprocess
 import sys
+import tempfile
 
 import pytest
 
@@ -23,7 +24,7 @@ KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "
 
 
 def _run(args, timeout=900):
-    env = dict(os.environ, MUON_BENCH_CLOCKS_DIR=os.path.join(ROOT, "gpurun_out"))
+    env = dict(os.environ, MUON_BENCH_CLOCKS_DIR=tempfile.mkdtemp(prefix="muon_bench_clocks_"))
     r = subprocess.run(args, cwd=ROOT, capture_output=True, text=True, timeout=timeout, env=env)
     assert r.returncode == 0, r.stderr[-3000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
