@@ -14,7 +14,8 @@
 // CTA pairs (clusters of 2 on one TPC) compute 256 x 256 output tiles with the
 // 2-SM MMA (tcgen05.mma.cta_group::2, M = 256, N = 256, K = 16): each CTA
 // stages its own 128 rows of the A operand and its half (128 rows) of the B
-// operand, so every SM reads 32 KB per 64-deep K step instead of 48 KB.
+// operand, so every SM reads 32 KB per 64-deep K step instead of 48 KB (16 KB
+// on the diagonal blocks of Gram and Poly, where the two operands coincide).
 // No TMA multicast is used; only the MMA commits arrive on both CTAs.
 //
 // Block layout (320 threads, one block per SM), in both CTAs of a pair:
