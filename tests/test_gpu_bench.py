@@ -49,6 +49,9 @@ def _check_common(d, steps):
     r = d["roofline"]
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert 0 < r["frac"] < 1.2 and r["achieved"] == pytest.approx(r["frac"] * r["peak"])
+    # a floor well under the ~0.5 of burst the chain reaches in short runs:
+    # a regression of the Newton-Schulz kernel fails here, not only in a number
+    assert r["frac"] > 0.35, r["frac"]
     assert r["flops_per_launch"] == pytest.approx(1.1421587866e12, rel=1e-9)
     assert d["gpu_launches"] == 4 * steps
 
