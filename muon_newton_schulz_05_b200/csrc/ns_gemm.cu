@@ -83,6 +83,20 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
   }
 }
 
+// Debug build: the boxes load_operand would copy lie inside their tensor map
+// (X maps: Cp columns x count*Rp rows; A and B maps: rp x count*rp). On a
+// violation the status word gets MUON_ERR_BOUNDS and the caller loads from
+// (0, 0) instead, so that the stage's bytes still arrive. Release build: true.
+__device__ __forceinline__ bool operand_in_bounds(const NsGemmParams& p, const BankPlan& bp, int slot,
+                                                  int mn_major, int base, int mn0, int k0) {
+  const bool x_map = slot == kHiK0 || slot == kHiK1 || slot == kHiMN0 || slot == kHiMN1;
+  const int64_t inner = x_map ? bp.Cp : bp.rp;
+  const int64_t outer = static_cast<int64_t>(bp.count) * (x_map ? bp.Rp : bp.rp);
+  const bool ok = mn_major ? (mn0 >= 0 && mn0 + 128 <= inner && base + k0 >= 0 && base + k0 + kBK <= outer)
+                           : (k0 >= 0 && k0 + kBK <= inner && base + mn0 >= 0 && base + mn0 + kBM <= outer);
+  return in_bounds(ok, p.status);
+}
+
 // Whether K block k0 of an operand whose rows start at mn0 is read
 // transposed: the operand is A or B and the 256-block (mn0, k0) lies below
 // the diagonal, so its values are those of the stored block (k0, mn0).
@@ -448,8 +462,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int tile = pair; ok && tile < ntiles; tile += npairs) {
         const Tile T = decode_tile(p, tile);
         if (T.phase == kReduce) continue;  // no MMA: the epilogue warps sum partials
-        const CUtensorMap* amap = &p.maps[T.bank][T.a_map];
-        const CUtensorMap* bmap = &p.maps[T.bank][T.b_map];
         // the operands of this tile are final once the phase it reads is done
         if (!wait_dependency(T.dep_cnt, T.dep_target, abort_flag, p.status, limit)) {
           ok = false;
@@ -471,11 +483,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const int k0 = (T.kb0 + kb) * kBK;
             const bool at = below_diagonal(T.a_sym, T.m0, k0);
             const bool bt = below_diagonal(T.b_sym, T.n0, k0);
-            load_operand(st, at ? &p.maps[T.bank][T.a_tmap] : amap, bar, at ? 1 : T.a_mn, T.a_base,
-                         T.m0 + kBM * rank, k0);
-            if (!T.same_ab)
-              load_operand(st + kATileBytes, bt ? &p.maps[T.bank][T.b_tmap] : bmap, bar, bt ? 1 : T.b_mn,
-                           T.b_base, T.n0 + (kBN / 2) * rank, k0);
+            const BankPlan& bp = p.bank[T.bank];
+            {
+              const int slot = at ? T.a_tmap : T.a_map, mn = at ? 1 : T.a_mn;
+              const int row = T.m0 + kBM * static_cast<int>(rank);
+              const bool ok = operand_in_bounds(p, bp, slot, mn, T.a_base, row, k0);
+              load_operand(st, &p.maps[T.bank][slot], bar, mn, ok ? T.a_base : 0, ok ? row : 0, ok ? k0 : 0);
+            }
+            if (!T.same_ab) {
+              const int slot = bt ? T.b_tmap : T.b_map, mn = bt ? 1 : T.b_mn;
+              const int row = T.n0 + (kBN / 2) * static_cast<int>(rank);
+              const bool ok = operand_in_bounds(p, bp, slot, mn, T.b_base, row, k0);
+              load_operand(st + kATileBytes, &p.maps[T.bank][slot], bar, mn, ok ? T.b_base : 0, ok ? row : 0,
+                           ok ? k0 : 0);
+            }
             issued_parity[stage] = static_cast<int>(phase);
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
