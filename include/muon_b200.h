@@ -44,8 +44,12 @@
  *     a checkpoint before resuming if the failed step must not count.
  *   - One Newton-Schulz chain is a persistent launch whose CTA pairs wait on
  *     one another; its grid is capped at the pairs the device can hold at
- *     once. Chains on several streams of one device are correct but
- *     serialise; kernels of other streams that hold SMs delay a chain.
+ *     once. Kernels of other streams that hold SMs only delay a chain, and
+ *     chains on streams of equal priority are dispatched in launch order and
+ *     serialise. A chain on a higher-priority stream can take SMs that an
+ *     earlier chain still needs; both then end with MUON_ERR_TIMEOUT (the
+ *     waits are bounded). Run one chain at a time per device, or give the
+ *     streams that carry steps the same priority.
  *   - Every device pointer must be 16-byte aligned. param, momentum,
  *     momentum_slow and ema are updated in place and must not overlap one
  *     another, in the same bank or in another bank of the call (checked:
