@@ -92,6 +92,22 @@ def test_orthogonalize_low_rank_gradients(rank, shape):
         assert sv_maxdiff(f64(out[0]), ref) <= TOL_SV
 
 
+@pytest.mark.parametrize("shape", [(1, 129, 257), (1, 768, 768), (1, 257, 129), (1, 256, 8192), (2, 384, 640)])
+def test_sixteen_steps_each_with_its_own_coefficients(shape):
+    """The most steps a call takes (16), each with different coefficients
+    (five quintic, then eleven convergent cubic variants with a + b = 1), so a
+    coefficient read from the wrong step shows: the same schedule shifted by
+    one step is 0.3 away from the oracle."""
+    s16 = [QUINTIC] * 5 + [(1.5 + 0.01 * j, -0.5 - 0.01 * j, 0.0) for j in range(11)]
+    cnt, R, C = shape
+    g = mi.gaussian(cnt * R, C, seed=R * 1000 + C, sigma=1.0).reshape(cnt, R, C).to(torch.bfloat16)
+    out = orth_gpu(g.to(DEV), s16).cpu()
+    for i in range(cnt):
+        ref = oracle.orthogonalize(f64(g[i]), s16, 1e-7)
+        assert rel_fro(f64(out[i]), ref) <= TOL_UPDATE, (i, rel_fro(f64(out[i]), ref))
+        assert sv_maxdiff(f64(out[i]), ref) <= TOL_SV
+
+
 def test_orthogonalize_bf16_output_and_fp32_input():
     x = mi.spiked_gaussian(768, 768, 5, 1e-3, 4, 10.0)[None].to(DEV)
     out = orth_gpu(x, [QUINTIC] * 5, out_dtype=torch.bfloat16)
