@@ -108,6 +108,22 @@ def test_sixteen_steps_each_with_its_own_coefficients(shape):
         assert sv_maxdiff(f64(out[i]), ref) <= TOL_SV
 
 
+def test_many_matrices_in_one_call():
+    """Hundreds of matrices in one call (thousands of tiles and per-matrix
+    counters in one persistent launch), wide and tall, every one checked.
+    The inputs are spiked like the benchmark banks' gradients (N(0, 1e-3^2)
+    plus a rank-4 spike at 10x RMS; a replay of the kernel's rounding puts
+    them at about half the tolerance; plain Gaussian matrices of this size
+    sit at 0.85-0.95 of it)."""
+    for base, cnt, R, C in ((1000, 300, 64, 128), (2000, 150, 128, 64)):
+        x = torch.stack([mi.spiked_gaussian(R, C, base + i, 1e-3, 4, 10.0) for i in range(cnt)])
+        out = orth_gpu(x.to(DEV), [QUINTIC] * 5).cpu()
+        for i in range(cnt):
+            ref = oracle.orthogonalize(f64(x[i]), [QUINTIC] * 5, 1e-7)
+            assert rel_fro(f64(out[i]), ref) <= TOL_UPDATE, (R, C, i, rel_fro(f64(out[i]), ref))
+            assert sv_maxdiff(f64(out[i]), ref) <= TOL_SV
+
+
 def test_orthogonalize_bf16_output_and_fp32_input():
     x = mi.spiked_gaussian(768, 768, 5, 1e-3, 4, 10.0)[None].to(DEV)
     out = orth_gpu(x, [QUINTIC] * 5, out_dtype=torch.bfloat16)
