@@ -50,6 +50,8 @@ NS_CHAIN_TRAFFIC = {
         "capture": "ncu --set full, one chain launch of the GPT-124M bank (second step)"},
     3: {"bytes": 4.876920e9, "source_sha16": "92c4d7963c97ccb8",
         "capture": "ncu --set full, one chain launch of the 64 x 1024^2 bank (second step)"},
+    5: {"bytes": 9.717949e9, "source_sha16": "92c4d7963c97ccb8",
+        "capture": "ncu --set full, one chain launch of the ANVIL bank with its 768 x 50304 readout (second step)"},
 }
 KERNEL_SOURCES = ("ns_gemm.cu", "plan.cuh", "ptx.cuh", "tiles.cuh")
 
