@@ -487,15 +487,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             {
               const int slot = at ? T.a_tmap : T.a_map, mn = at ? 1 : T.a_mn;
               const int row = T.m0 + kBM * static_cast<int>(rank);
-              const bool ok = operand_in_bounds(p, bp, slot, mn, T.a_base, row, k0);
-              load_operand(st, &p.maps[T.bank][slot], bar, mn, ok ? T.a_base : 0, ok ? row : 0, ok ? k0 : 0);
+              const bool in_map = operand_in_bounds(p, bp, slot, mn, T.a_base, row, k0);
+              load_operand(st, &p.maps[T.bank][slot], bar, mn, in_map ? T.a_base : 0, in_map ? row : 0,
+                           in_map ? k0 : 0);
             }
             if (!T.same_ab) {
               const int slot = bt ? T.b_tmap : T.b_map, mn = bt ? 1 : T.b_mn;
               const int row = T.n0 + (kBN / 2) * static_cast<int>(rank);
-              const bool ok = operand_in_bounds(p, bp, slot, mn, T.b_base, row, k0);
-              load_operand(st + kATileBytes, &p.maps[T.bank][slot], bar, mn, ok ? T.b_base : 0, ok ? row : 0,
-                           ok ? k0 : 0);
+              const bool in_map = operand_in_bounds(p, bp, slot, mn, T.b_base, row, k0);
+              load_operand(st + kATileBytes, &p.maps[T.bank][slot], bar, mn, in_map ? T.b_base : 0,
+                           in_map ? row : 0, in_map ? k0 : 0);
             }
             issued_parity[stage] = static_cast<int>(phase);
           }
