@@ -209,8 +209,10 @@ muon_status muon_device_status(void* ws, size_t ws_bytes, void* stream, int32_t 
 muon_status muon_set_ns_events(void* before_ns, void* after_ns);
 
 /* Host only, no GPU needed: the Newton-Schulz chain's tile list for banks of
- * the given shapes (shapes[3b..3b+2] = count, rows, cols of bank b) and
- * ns_steps, as the kernel decodes it. Tiles are listed step by step, phase by
+ * the given shapes and ns_steps, as the kernel decodes it (for tests and
+ * tooling). shapes: host array of 3 * nbanks values, (count, rows, cols) of
+ * bank b at shapes[3b..3b+2], validated like a step's banks. tiles: host array
+ * owned by the caller, or NULL to only count. Tiles are listed step by step, phase by
  * phase (Gram, Reduce, Poly, Apply), bank by bank, matrix by matrix. If
  * tiles_cap >= 13 * (number of tiles), tiles[13t..13t+12] = (step, phase
  * (0 Gram, 1 Poly, 2 Apply, 3 Reduce), bank, matrix, first output row, first
