@@ -243,13 +243,33 @@ def _oracle_layers(w):
     return 1 if w.n_params > 1_000_000_000 else None
 
 
+REFERENCE_BUDGET_S = 180.0   # the reference arm's whole run, warm-up included
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     w = _workload(args.workload)
     layers = _oracle_layers(w)
-    for s in range(args.warmup):
+    # One untimed step over the (capped) bank first: if the requested steps
+    # would not fit the budget at that rate, every later step times the first
+    # `layers` matrices of each shape instead and scales them by the bank's
+    # counts (labelled as a sample in the line).
+    t_probe, _ = _oracle_bank_time(w, 0, layers)
+    remaining = args.steps + max(args.warmup - 1, 0)
+    budget = max(REFERENCE_BUDGET_S - t_probe, 0.0)
+    if remaining and t_probe * remaining > budget:
+        # a matrix's oracle time goes with its Newton-Schulz work, R C min(R, C)
+        def work(cap):
+            return sum(min(sp.count, cap) * sp.rows * sp.cols * min(sp.rows, sp.cols) for sp in w.banks)
+        most = max(sp.count for sp in w.banks) if layers is None else layers
+        full = work(most)
+        cap = most
+        while cap > 1 and t_probe * work(cap) / full * remaining > budget:
+            cap -= 1
+        layers = cap
+    for s in range(1, args.warmup):
         _oracle_bank_time(w, s, layers)
     times = []
     desc = ""

@@ -64,3 +64,33 @@ def test_source_hash_ignores_comments():
     assert bench.code_only(a) == bench.code_only(b)
     assert bench.code_only(a) != bench.code_only(a.replace("2 * x", "3 * x"))
     assert bench.chain_traffic(2)[0] is not None   # the stored capture describes these sources
+
+
+def test_reference_arm_fits_its_budget(monkeypatch, capsys):
+    """The reference arm times the whole bank each step when the requested
+    steps fit its time budget, and otherwise the first matrices of each shape
+    (scaled, labelled) so that the run still ends in a few minutes. A fake
+    oracle timer stands in for the float64 oracle: 6 s per whole GPT bank,
+    each matrix's share proportional to R C min(R, C)."""
+    import json
+    import types
+    calls = []
+
+    def fake(w, step=0, max_layers=None):
+        def work(cap):
+            return sum((sp.count if cap is None else min(sp.count, cap)) * sp.rows * sp.cols
+                       * min(sp.rows, sp.cols) for sp in w.banks)
+        t = 6.0 * work(max_layers) / work(None)
+        calls.append((max_layers, t, f"sample {max_layers}"))
+        return t, calls[-1][2]
+    monkeypatch.setattr(bench, "_oracle_bank_time", fake)
+    for steps, warmup, whole in ((20, 5, True), (200, 10, False)):
+        calls.clear()
+        bench.run_reference(types.SimpleNamespace(workload=2, steps=steps, warmup=warmup, gpus=1))
+        line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+        assert line["steps"] == steps and line["impl"] == "reference"
+        assert len(calls) == steps + max(warmup, 1)
+        run_s = sum(c[1] for c in calls)
+        assert run_s <= bench.REFERENCE_BUDGET_S, run_s
+        assert (calls[-1][0] is None) == whole
+        assert line["cpu_baseline"]["sample"].endswith(calls[-1][2])
