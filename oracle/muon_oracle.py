@@ -51,7 +51,7 @@ rational orbits and the page constants); none is "parity unpinned".
 from __future__ import annotations
 
 import math
-from typing import Iterable, Sequence
+from typing import Sequence
 
 import numpy as np
 
@@ -307,14 +307,3 @@ def ns_flops_algorithmic(rows: int, cols: int, steps: int) -> float:
     r, c = min(rows, cols), max(rows, cols)
     return float(steps) * (r * (r + 1) * c + r * r * (r + 1) + 2.0 * r * r * c)
 
-
-def bank_muon_step(thetas: Iterable, grads: Iterable, moms: Iterable, hp: dict,
-                   param_dtype: str):
-    """muon_step over a list of matrices (plain loop)."""
-    out_t, out_m, out_o = [], [], []
-    for th, g, m in zip(thetas, grads, moms):
-        t1, m1, o1 = muon_step(th, g, m, hp, param_dtype)
-        out_t.append(t1)
-        out_m.append(m1)
-        out_o.append(o1)
-    return out_t, out_m, out_o

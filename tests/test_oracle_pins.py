@@ -10,8 +10,12 @@
   * Invariants: transpose, gradient scale, permutations, G = 0, rank one.
   * The page constants in tests/golden/pages_constants.json.
   * bf16 rounding against torch's float32 -> bfloat16 conversion.
+  * Whole-step closed forms: rank one (Muon), diagonal matrices (SGD form,
+    with and without Nesterov), tall rank one with zero rows (ANVIL).
+  * The flop count against a count of a small case's multiply-adds.
   * Sensitivity: plausible mistakes (wrong sign, dropped term, transposed
-    Gram) make the closed-form pin fail.
+    Gram) make the closed-form pin fail; test_oracle_mutants plants one-line
+    mistakes in every function and names the pin that catches each.
 """
 import json
 import math
@@ -156,6 +160,32 @@ def test_sgd_form_three_step_unroll_and_step():
     assert np.array_equal(t_sg, t_ma)
 
 
+@pytest.mark.parametrize("nesterov", [0, 1])
+def test_sgd_form_step_on_diagonal_matrices_closed_form(nesterov):
+    """On 'diagonal' 4 x 6 matrices every product of the iteration stays
+    diagonal, so O is the scalar orbit of each entry of U / ||U||_F. From a
+    momentum that is not a multiple of the gradient the SGD form gives
+    M' = mu M + G and U = G + mu M' with Nesterov (else U = M'): two
+    directions the normalisation cannot make equal."""
+    def diag(d):
+        return np.eye(4, 6) * d[:, None]
+
+    g = np.array([1.0, -2.0, 0.5, 3.0])
+    m0 = np.array([4.0, 1.0, -2.0, 0.5])
+    mu, lr, wd = 0.9, 0.02, 0.3
+    th = np.arange(24, dtype=np.float64).reshape(4, 6) / 10.0
+    hp = dict(lr=lr, mu=mu, weight_decay=wd, nesterov=nesterov, coeffs=[QUINTIC] * 5, eps=0.0,
+              sgd_momentum=1)
+    t1, M1, O = oracle.muon_step(th, diag(g), diag(m0), hp, "f32")
+    m1 = mu * m0 + g
+    u = g + mu * m1 if nesterov else m1
+    assert np.max(np.abs(M1 - diag(m1))) < 1e-15
+    O_exp = diag(_scalar_orbit(u / np.linalg.norm(u), [QUINTIC] * 5))
+    assert np.max(np.abs(O - O_exp)) < 1e-12
+    th_exp = th * (1 - lr * wd) - lr * 1.0 * O_exp
+    assert np.max(np.abs(t1 - th_exp)) <= 1e-6 * np.max(np.abs(th_exp))
+
+
 def test_sgd_momentum_form_gives_the_same_update():
     """From zero state the SGD form M' = mu M' + G is M / (1 - mu); the
     normalisation removes the factor, so O is the same (reading R1)."""
@@ -278,6 +308,34 @@ def test_cautious_mask_closed_form():
     assert np.max(np.abs(t1 - expect)) < 1e-6
 
 
+def test_anvil_tall_rank_one_with_zero_rows_closed_form():
+    """A tall rank-one gradient G = u v^T with two exactly-zero rows, both
+    momenta starting at zero: Mf = (1 - beta_fast) G, Ms = (1 - beta_slow) G,
+    O = p^6(s0) u^ v^T, so O * Ms > 0 wherever G != 0 and is exactly 0 on the
+    zero rows. The sign-agreement rule is strict there (no sign, no decay):
+    those rows of theta come back unchanged. Elsewhere theta decays and takes
+    the update scaled by max(1, R/C)^(1/2) = 2 for a 12 x 3 matrix."""
+    rows, cols = 12, 3
+    rng = np.random.default_rng(1203)
+    u = rng.standard_normal(rows)
+    u[[4, 9]] = 0.0
+    v = rng.uniform(0.5, 1.5, cols) * np.array([1.0, -1.0, 1.0])
+    G = np.outer(u, v)
+    th = rng.standard_normal((rows, cols))
+    lr, wd, bf, bs, eps = 0.05, 0.4, 0.9, 0.99, 1e-7
+    hp = dict(lr=lr, beta_fast=bf, beta_slow=bs, weight_decay=wd, coeffs=[QUINTIC] * 6, eps=eps)
+    t1, Mf, Ms, O, mask = oracle.anvil_step(th, G, np.zeros_like(G), np.zeros_like(G), hp, "f32")
+    nrm = (1 - bf) * np.linalg.norm(u) * np.linalg.norm(v)
+    p = _scalar_orbit([nrm / (nrm + eps)], [QUINTIC] * 6)[0]
+    assert p > 0
+    O_exp = p * np.outer(u / np.linalg.norm(u), v / np.linalg.norm(v))
+    assert np.max(np.abs(O - O_exp)) < 1e-12
+    assert np.array_equal(mask, (G != 0).astype(float))
+    th_exp = np.where(G != 0, th * (1 - lr * wd), th) - lr * 2.0 * O_exp
+    assert np.array_equal(t1[[4, 9]], th[[4, 9]].astype(np.float32).astype(np.float64))
+    assert np.max(np.abs(t1 - th_exp)) <= 1e-6 * np.max(np.abs(th_exp))
+
+
 def test_round_to_bf16_matches_torch():
     rng = np.random.default_rng(0)
     x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-20, 20, 20000),
@@ -294,6 +352,23 @@ def test_flop_count_matches_dense_count_minus_symmetry():
     assert f == oracle.ns_flops_algorithmic(r, c, 1)
     dense = 4 * r * r * c + 2 * r ** 3
     assert f < dense and f > 0.7 * dense
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (3, 5), (4, 4), (7, 2)])
+def test_flop_count_by_counting_operations(shape):
+    """Count the multiply-adds one iteration performs when A = X X^T and
+    A A are computed on and above the diagonal only (each entry a dot
+    product of length c, resp. r) and B X in full, two flops each."""
+    r, c = min(shape), max(shape)
+    flops = 0
+    for i in range(r):
+        for j in range(i, r):
+            flops += 2 * c          # A_ij = <x_i, x_j>
+            flops += 2 * r          # (A A)_ij
+    for i in range(r):
+        for j in range(c):
+            flops += 2 * r          # (B X)_ij
+    assert oracle.ns_flops_algorithmic(*shape, 3) == 3 * flops
 
 
 # ---- sensitivity: plausible mistakes must break the closed-form pin -------
