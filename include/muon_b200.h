@@ -54,6 +54,12 @@
  *     momentum_slow and ema are updated in place and must not overlap one
  *     another, in the same bank or in another bank of the call (checked:
  *     MUON_ERR_ALIAS), nor the workspace (not checked); grad is read only.
+ *   - Size limits (MUON_ERR_SHAPE beyond them): rows and cols, rounded up
+ *     to 256, below 2^24; per bank, count times the rounded rows below 2^31,
+ *     and below 2^30 its 256 x 256 output tiles and its 8192-element blocks;
+ *     over all banks of a call, the chain's tiles (every phase, times
+ *     ns_steps) and the elementwise blocks below 2^31: the kernels index
+ *     them with 32-bit integers.
  */
 #ifndef MUON_B200_H
 #define MUON_B200_H

@@ -276,6 +276,23 @@ UpdBank update_io(const muon_bank& b, const muon_hparams* hp) {
 
 // Tile prefix sums of the chain (list order: step, phase Gram / Reduce / Poly
 // / Apply, bank, matrix).
+// check_shape bounds each bank on its own; the chain numbers its tiles (over
+// every bank, phase and step) and the momentum and update passes their blocks
+// (over every bank) with 32-bit ints, so those totals must stay below 2^31.
+muon_status check_totals(const Shape3* shapes, int nbanks, int ns_steps) {
+  BankPlan plans[MUON_MAX_BANKS];
+  plan_workspace(shapes, nbanks, nullptr, plans);
+  int64_t tiles = 0, blocks = 0;
+  for (int b = 0; b < nbanks; ++b) {
+    const BankPlan& p = plans[b];
+    tiles += static_cast<int64_t>(p.count) *
+             (static_cast<int64_t>(p.tiles_sym) * p.ksplit + p.tiles_red + p.tiles_sym + p.tiles_apply);
+    blocks += static_cast<int64_t>(p.count) * p.chunks;
+  }
+  const int64_t lim = int64_t(1) << 31;
+  return (tiles * ns_steps >= lim || blocks >= lim) ? MUON_ERR_SHAPE : MUON_OK;
+}
+
 void plan_chain(NsGemmParams& gp, const BankPlan* plans, int nbanks) {
   gp.nbanks = nbanks;
   int gram = 0, red = 0, sym = 0, app = 0;
@@ -393,6 +410,9 @@ muon_status check_common(const muon_bank* banks, int32_t nbanks, const muon_hpar
   muon_status st = check_banks(banks, nbanks, anvil);
   if (st != MUON_OK) return st;
   if ((st = check_ns(hp)) != MUON_OK) return st;
+  Shape3 shapes[MUON_MAX_BANKS];
+  for (int b = 0; b < nbanks; ++b) shapes[b] = {banks[b].count, banks[b].rows, banks[b].cols};
+  if ((st = check_totals(shapes, nbanks, hp->ns_steps)) != MUON_OK) return st;
   if (!finite(hp->lr) || !finite(hp->weight_decay) || hp->weight_decay < 0.0f) return MUON_ERR_HPARAM;
   if (anvil) {
     if (!beta_ok(hp->beta_fast) || !beta_ok(hp->beta_slow)) return MUON_ERR_HPARAM;
@@ -466,6 +486,8 @@ muon_status muon_orthogonalize(const void* in, int32_t in_dtype, void* out, int3
   if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return MUON_ERR_DTYPE;
   if (!aligned16(in) || !aligned16(out)) return MUON_ERR_ALIGN;
   if ((st = check_ns(hp)) != MUON_OK) return st;
+  const Shape3 one = {count, rows, cols};
+  if ((st = check_totals(&one, 1, hp->ns_steps)) != MUON_OK) return st;
   if (!ws) return MUON_ERR_WORKSPACE;
   if (!aligned16(ws)) return MUON_ERR_ALIGN;
   muon_bank bank;
@@ -489,7 +511,7 @@ muon_status ema_update(const muon_bank* banks, int32_t nbanks, float beta, void*
   for (int b = 0; b < nbanks; ++b) {
     const muon_bank& k = banks[b];
     if (!k.ema) continue;
-    if (k.count < 1 || k.rows < 1 || k.cols < 1) return MUON_ERR_SHAPE;
+    if (check_shape(k.count, k.rows, k.cols) != MUON_OK) return MUON_ERR_SHAPE;
     if (!k.param) return MUON_ERR_NULL;
     if (!dtype_ok(k.param_dtype)) return MUON_ERR_DTYPE;
     if (!aligned16(k.param) || !aligned16(k.ema)) return MUON_ERR_ALIGN;
@@ -575,6 +597,8 @@ muon_status muon_orthogonalize_static(const void* in, int32_t in_dtype, void* ou
   if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return MUON_ERR_DTYPE;
   if (!aligned16(in) || !aligned16(out)) return MUON_ERR_ALIGN;
   if ((st = check_ns(hp)) != MUON_OK) return st;
+  const Shape3 one = {count, rows, cols};
+  if ((st = check_totals(&one, 1, hp->ns_steps)) != MUON_OK) return st;
   muon_bank bank;
   std::memset(&bank, 0, sizeof(bank));
   bank.count = count;
@@ -613,6 +637,8 @@ int64_t muon_chain_plan(const int64_t* shapes, int32_t nbanks, int32_t ns_steps,
     const muon_status st = check_shape(sh[b].count, sh[b].rows, sh[b].cols);
     if (st != MUON_OK) return -static_cast<int64_t>(st);
   }
+  const muon_status tot = check_totals(sh, nbanks, ns_steps);
+  if (tot != MUON_OK) return -static_cast<int64_t>(tot);
   static thread_local NsGemmParams gp;  // large; kept off the stack
   std::memset(&gp, 0, sizeof(gp));
   BankPlan plans[MUON_MAX_BANKS];

@@ -228,3 +228,57 @@ def test_checkpoint_average_betas_match_the_oracle():
         mb.checkpoint_average_betas([0.0, 1.0])
     with pytest.raises(ValueError):
         mb.checkpoint_average_betas([1.0, -1.0])
+
+
+HUGE = dict(count=500000, rows=4096, cols=4096)   # passes the per-bank shape check
+
+
+def _plan_count(shapes, ns_steps):
+    lib = mb.raw_library()
+    f = lib.muon_chain_plan
+    f.restype = ctypes.c_int64
+    sh = (ctypes.c_int64 * (3 * len(shapes)))(*[v for s in shapes for v in s])
+    return f(sh, len(shapes), ns_steps, None, ctypes.c_int64(0))
+
+
+def test_totals_over_banks_and_steps_stay_in_32_bits():
+    """Each bank can pass its own shape check while the chain's tile count over
+    all phases and steps, or the elementwise passes' block count over all
+    banks, would not fit the kernels' 32-bit indices: those are refused too."""
+    one = (HUGE["count"], HUGE["rows"], HUGE["cols"])
+    # 500000 x (136 Gram + 136 Poly + 256 Apply) tiles per step
+    assert _plan_count([one], 5) == 5 * 500000 * 528
+    assert _plan_count([one], 16) == -2
+    # 500000 x 2048 momentum blocks per bank: two banks fit, three do not
+    assert _plan_count([one] * 2, 1) == 2 * 500000 * 528
+    assert _plan_count([one] * 3, 1) == -2
+
+
+@pytest.mark.parametrize("fn", ["muon_step", "anvil_step"])
+def test_step_refuses_totals_beyond_32_bits_before_the_workspace_check(fn):
+    spaced = dict(param=1 << 48, grad=2 << 48, momentum=3 << 48,
+                  momentum_slow=(4 << 48) if fn == "anvil_step" else None)
+    bank = _bank(**HUGE, **spaced)
+    q = (3.4445, -4.7750, 2.0315)
+    assert _call(fn, bank, hp=mb.Hparams(coeffs=[q] * 5)) == 6        # only the workspace is short
+    assert _call(fn, bank, hp=mb.Hparams(coeffs=[q] * 16)) == 2       # 16 steps: too many tiles
+
+
+def test_orthogonalize_refuses_totals_beyond_32_bits():
+    lib = mb.raw_library()
+    q = (3.4445, -4.7750, 2.0315)
+    for steps, want in ((5, 6), (16, 2)):
+        h = mb.Hparams(coeffs=[q] * steps).to_c()
+        st = lib.muon_orthogonalize(ctypes.c_void_p(1 << 48), mb.BF16, ctypes.c_void_p(2 << 48), mb.F32,
+                                    ctypes.c_int64(HUGE["count"]), ctypes.c_int64(HUGE["rows"]),
+                                    ctypes.c_int64(HUGE["cols"]), ctypes.byref(h),
+                                    ctypes.c_void_p(FAKE), ctypes.c_size_t(1 << 30), None)
+        assert st == want, (steps, st)
+
+
+def test_ema_update_bounds_the_shape_before_multiplying():
+    lib = mb.raw_library()
+    for kw in (dict(count=1 << 40), dict(rows=1 << 40, cols=1 << 40), dict(count=0)):
+        b = _bank(ema=FAKE + 0x4000, **kw)
+        arr = (mb.CBank * 1)(b)
+        assert lib.ema_update(arr, 1, ctypes.c_float(0.9), None) == 2, kw
