@@ -274,8 +274,6 @@ UpdBank update_io(const muon_bank& b, const muon_hparams* hp) {
   return UpdBank{b.param, b.param_dtype, b.momentum_slow, b.ema, static_cast<float>(double(hp->lr) * s)};
 }
 
-// Tile prefix sums of the chain (list order: step, phase Gram / Reduce / Poly
-// / Apply, bank, matrix).
 // check_shape bounds each bank on its own; the chain numbers its tiles (over
 // every bank, phase and step) and the momentum and update passes their blocks
 // (over every bank) with 32-bit ints, so those totals must stay below 2^31.
@@ -293,6 +291,8 @@ muon_status check_totals(const Shape3* shapes, int nbanks, int ns_steps) {
   return (tiles * ns_steps >= lim || blocks >= lim) ? MUON_ERR_SHAPE : MUON_OK;
 }
 
+// Tile prefix sums of the chain (list order: step, phase Gram / Reduce / Poly
+// / Apply, bank, matrix).
 void plan_chain(NsGemmParams& gp, const BankPlan* plans, int nbanks) {
   gp.nbanks = nbanks;
   int gram = 0, red = 0, sym = 0, app = 0;
